@@ -1,0 +1,459 @@
+#!/usr/bin/env python
+"""Decode-attention benchmark for libdcp (sequence-sharded paged KV cache).
+
+One step = one pass of the whole hot path over the batch, for one new token
+per request:
+  dcp_shard_map (owner/slot of position L_b)  ->  dcp_kv_append (write the new
+  token into its owner's page)  ->  dcp_decode_partial (all N shards' partial
+  attention over positions [0, L_b + 1))  ->  dcp_merge (LSE merge).
+Lengths grow by one token per step, as in decoding.
+
+Metric: KV GB/s = (sum_b attended tokens x KV bytes per token) / step time,
+plus decode steps/s, and the fraction of the measured HBM copy bandwidth.
+Inputs are synthetic (seeded generator) with the shapes of the named
+workload; the KV cache (>= several GB) is far larger than the 126 MB L2, so
+no L2 flush is needed between steps.
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--config 5]
+                  [--n-shards 8] [--interleave 1] [--impl ours|reference]
+
+Multi-GPU (torchrun, one rank per GPU): each rank runs its own independent
+batch (replicas of the workload, weak scaling); there is no data-path
+collective.  Timing is the max over ranks of the device time.
+"""
+from __future__ import annotations
+
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import numpy as np
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import synth  # noqa: E402
+
+METRIC = "DCP decode-attn KV GB/s (% of B200 HBM peak) and decode steps/s per config"
+HEADLINE_CONFIG = 5
+
+
+def parse():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--config", type=int, default=HEADLINE_CONFIG)
+    ap.add_argument("--n-shards", type=int, default=None)
+    ap.add_argument("--interleave", type=int, default=None)
+    ap.add_argument("--batch-limit", type=int, default=None,
+                    help="keep only the first B requests of the workload (small profiling cases)")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU work of the oracle sample")
+    return ap.parse_args()
+
+
+def peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        d = json.load(open(p))
+        return float(d["hbm_gbs"]), "measured"
+    return 6650.0, "fallback"
+
+
+def get_workload(args):
+    w = synth.workload(args.config, n_shards=args.n_shards, interleave=args.interleave)
+    if args.batch_limit:
+        w.B = min(w.B, args.batch_limit)
+        w.lengths = w.lengths[:w.B]
+    return w
+
+
+def workload_config(w, args):
+    return {"workload": f"config{args.config}: {w.name}", "kind": w.kind, "kv_dtype": w.dtype,
+            "batch": w.B, "q_heads": w.hq, "kv_heads": w.hkv, "dk": w.dk, "dv": w.dv, "page_size": w.page_size,
+            "n_shards": w.n_shards, "interleave": w.interleave, "total_tokens": int(np.sum(w.lengths)),
+            "median_len": int(np.median(w.lengths)), "max_len": int(np.max(w.lengths)),
+            "l2": "inputs larger than L2 (KV cache >> 126 MB); no flush"}
+
+
+# ----------------------------------------------------------------------------
+# clocks sampling during the timed region
+# ----------------------------------------------------------------------------
+
+class Clocks:
+    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+         "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+         "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+        self.p = None
+
+    def start(self):
+        try:
+            self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
+                                       "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                      stderr=subprocess.DEVNULL)
+        except (OSError, FileNotFoundError):
+            self.p = None
+
+    def stop(self):
+        if self.p is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        self.p.terminate()
+        try:
+            self.p.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.p.kill()
+        self.f.flush()
+        rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
+        os.unlink(self.f.name)
+        sm, mx, reasons = [], None, set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            r = [x.strip() for x in r]
+            if len(r) < 9:
+                continue
+            try:
+                sm.append(float(r[1]))
+                mx = float(r[2])
+            except ValueError:
+                continue
+            for nm, v in zip(names, r[5:9]):
+                if v.lower() == "active":
+                    reasons.add(nm)
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "samples": len(sm),
+                "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------
+# our implementation
+# ----------------------------------------------------------------------------
+
+def run_ours(args, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    import sequence_sharded_paged_b200 as dcp
+    import synth.device as sdev
+    from sequence_sharded_paged_b200 import workload as wl
+
+    dcp.lib()  # fail loudly if libdcp.so is missing
+    torch.cuda.set_device(local_rank)
+    dev = torch.device("cuda", local_rank)
+    w = get_workload(args)
+    w.seed_val += 100 * rank  # each rank decodes its own independent batch
+    E = 0 if args.no_e2e else args.steps
+    growth = args.warmup + args.steps + E + 1
+    counts = wl.gpu_shard_counts(np.asarray(w.lengths) + growth, w.n_shards, w.interleave)
+    t0 = time.time()
+    dw = wl.build(w, counts)
+    fill_s = time.time() - t0
+    B, N = w.B, w.n_shards
+    L0 = torch.as_tensor(np.asarray(w.lengths, np.int32), device=dev)
+
+    n_total = args.warmup + args.steps + E
+    # per-step inputs, resident in HBM before the timed region
+    qs = [sdev.q(w.seed_val, B, w.hq, w.dk, step=s + 1) for s in range(n_total)]
+    req = torch.arange(B, dtype=torch.int32, device=dev)
+    pos_s = [(L0 + s).contiguous() for s in range(n_total)]
+    lens_s = [(L0 + s + 1).contiguous() for s in range(n_total)]
+    if w.kind == "gqa":
+        new_rows = [sdev.gqa_rows(w.seed_val, req, pos_s[s], w.hkv, w.dk) for s in range(n_total)]
+    else:
+        new_rows = [(sdev.latent_rows(w.seed_val, req, pos_s[s]), None) for s in range(n_total)]
+    rank_o = torch.empty(B, dtype=torch.int32, device=dev)
+    local_o = torch.empty(B, dtype=torch.int32, device=dev)
+    slot_o = torch.empty(B, dtype=torch.int64, device=dev)
+    o_part = torch.empty((N, B, w.hq, w.dv), dtype=torch.float32, device=dev)
+    lse = torch.empty((N, B, w.hq), dtype=torch.float32, device=dev)
+    out = torch.empty((B, w.hq, w.dv), dtype=torch.float32, device=dev)
+    lse_out = torch.empty((B, w.hq), dtype=torch.float32, device=dev)
+    stream = torch.cuda.current_stream()
+
+    def step(s, ev=None):
+        dcp.dcp_shard_map(dw.desc, pos_s[s], None, rank_o, local_o, slot_o)
+        k, v = new_rows[s]
+        dcp.dcp_kv_append(dw.desc, None, pos_s[s], k, v)
+        if ev is not None:
+            ev[0].record(stream)
+        dcp.dcp_decode_partial(dw.desc, qs[s], lens_s[s], o_part, lse, dw.ws)
+        if ev is not None:
+            ev[1].record(stream)
+        dcp.dcp_merge(o_part, lse, out, lse_out)
+
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    st = dcp.dcp_get_device_status()
+    if st != dcp.DCP_OK:
+        raise RuntimeError(f"device status after warm-up: {dcp.status_string(st)}")
+
+    kv_tok = [int(np.sum(w.lengths)) + B * (s + 1) for s in range(n_total)]
+    bpt = w.kv_bytes_per_token
+    ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
+    t_start = torch.cuda.Event(enable_timing=True)
+    t_stop = torch.cuda.Event(enable_timing=True)
+    clocks = Clocks(local_rank)
+    if world > 1:
+        dist.barrier()
+    torch.cuda.synchronize()
+    clocks.start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i, ev_k[i])
+    t_stop.record(stream)
+    torch.cuda.synchronize()
+    if world > 1:
+        dist.barrier()
+    clk = clocks.stop()
+    st = dcp.dcp_get_device_status()
+    if st != dcp.DCP_OK:
+        raise RuntimeError(f"device status after timed steps: {dcp.status_string(st)}")
+    ms = t_start.elapsed_time(t_stop)
+    kern_ms = [a.elapsed_time(b) for a, b in ev_k]
+    bytes_timed = sum(kv_tok[args.warmup + i] for i in range(args.steps)) * bpt
+
+    # end to end through the C ABI with host buffers: H2D of the step's inputs
+    # (q, new token rows, positions, lengths) from pinned memory, D2H of out + lse
+    e2e = None
+    if E:
+        pin = []
+        for s in range(args.warmup + args.steps, n_total):
+            k, v = new_rows[s]
+            pin.append((qs[s].cpu().pin_memory(), k.cpu().pin_memory(), None if v is None else v.cpu().pin_memory(),
+                        pos_s[s].cpu().pin_memory(), lens_s[s].cpu().pin_memory()))
+        q_d, k_d = torch.empty_like(qs[0]), torch.empty_like(new_rows[0][0])
+        v_d = None if new_rows[0][1] is None else torch.empty_like(new_rows[0][1])
+        pos_d, len_d = torch.empty_like(pos_s[0]), torch.empty_like(lens_s[0])
+        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
+        lse_h = torch.empty(lse_out.shape, dtype=lse_out.dtype).pin_memory()
+        h2d = sum(t.numel() * t.element_size() for t in pin[0] if t is not None)
+        d2h = out_h.numel() * 4 + lse_h.numel() * 4
+        e0 = torch.cuda.Event(enable_timing=True)
+        e1 = torch.cuda.Event(enable_timing=True)
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+        e0.record(stream)
+        for i, (qh, kh, vh, ph, lh) in enumerate(pin):
+            q_d.copy_(qh, non_blocking=True)
+            k_d.copy_(kh, non_blocking=True)
+            if vh is not None:
+                v_d.copy_(vh, non_blocking=True)
+            pos_d.copy_(ph, non_blocking=True)
+            len_d.copy_(lh, non_blocking=True)
+            dcp.dcp_shard_map(dw.desc, pos_d, None, rank_o, local_o, slot_o)
+            dcp.dcp_kv_append(dw.desc, None, pos_d, k_d, v_d)
+            dcp.dcp_decode_partial(dw.desc, q_d, len_d, o_part, lse, dw.ws)
+            dcp.dcp_merge(o_part, lse, out, lse_out)
+            out_h.copy_(out, non_blocking=True)
+            lse_h.copy_(lse_out, non_blocking=True)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        if world > 1:
+            dist.barrier()
+        e2e_ms = e0.elapsed_time(e1)
+        e2e_bytes = sum(kv_tok[args.warmup + args.steps + i] for i in range(E)) * bpt
+        e2e = (e2e_ms, e2e_bytes, h2d, d2h)
+
+    # max over ranks of device time; whole-job bytes
+    if world > 1:
+        t = torch.tensor([ms, sum(kern_ms), e2e[0] if e2e else 0.0], device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms, kern_total, e2e_ms_max = t.tolist()
+        tb = torch.tensor([float(bytes_timed), float(e2e[1] if e2e else 0)], device=dev, dtype=torch.float64)
+        dist.all_reduce(tb, op=dist.ReduceOp.SUM)
+        bytes_all, e2e_bytes_all = tb.tolist()
+    else:
+        kern_total = sum(kern_ms)
+        bytes_all = float(bytes_timed)
+        e2e_ms_max = e2e[0] if e2e else 0.0
+        e2e_bytes_all = float(e2e[1]) if e2e else 0.0
+
+    hbm, peak_kind = peaks()
+    gbs = bytes_all / (ms * 1e-3) / 1e9
+    # dominant kernel: the decode (plan + split-KV attention) of one step, CUDA events on its stream
+    per_launch_bytes = bytes_timed / args.steps
+    kern_avg_ms = kern_total / args.steps
+    achieved = per_launch_bytes / (kern_avg_ms * 1e-3) / 1e9
+    res = {
+        "metric": METRIC,
+        "value": round(gbs, 1),
+        "unit": "GB/s",
+        "n_gpus": world,
+        "steps": args.steps,
+        "warmup": args.warmup,
+        "ms_per_step": round(ms / args.steps, 4),
+        "steps_per_s": round(args.steps / (ms * 1e-3), 2),
+        "pct_hbm_measured": round(100 * gbs / world / hbm, 1),
+        "pct_hbm_nominal_8tbs": round(100 * gbs / world / 8000.0, 1),
+        "higher_is_better": True,
+        "scaling": "weak",
+        "vs_baseline": None,
+        "dtype": "bf16" if w.dtype == "bf16" else "fp8_e4m3 cache, bf16 q, fp32 accumulate",
+        "data": "synthetic (seeded counter-based generator; lengths shaped like the agentic trace)",
+        "config": workload_config(w, args) | {"parallelism": f"replicas x{world} (one independent batch per GPU)"},
+        "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(achieved / hbm, 3), "traffic": None,
+                     "kernel": "dcp_decode_partial (planner + split-KV attention)",
+                     "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
+                     else "fallback 6650 GB/s"},
+        "clocks": clk,
+        "gpu_launches": 5 * args.steps,
+        "fill_seconds": round(fill_s, 2),
+    }
+    if e2e:
+        res["e2e"] = {"value": round(e2e_bytes_all / (e2e_ms_max * 1e-3) / 1e9, 1), "unit": "GB/s",
+                      "h2d_bytes_per_step": e2e[2], "d2h_bytes_per_step": e2e[3],
+                      "ms_per_step": round(e2e_ms_max / E, 4)}
+    return res, w
+
+
+# ----------------------------------------------------------------------------
+# the oracle on host cores (CPU baseline / reference arm)
+# ----------------------------------------------------------------------------
+
+def oracle_sample(w, cpu_seconds: float, rate_tok_s: float | None = None):
+    """Pick requests (shortest-first from a seeded shuffle) until the sample
+    holds about cpu_seconds of oracle work; returns (req_list, tokens)."""
+    # calibrated oracle throughput (tokens*heads per second per core, float64 two-pass)
+    import oracle
+    cores = oracle.num_threads()
+    per_tok = (w.hq * (w.dk + w.dv) * 2) if w.kind == "mla" else (w.hq * (w.dk + w.dv) * 2)
+    flops_s = 1.0e9 * cores if rate_tok_s is None else rate_tok_s
+    budget_tok = max(1000, int(cpu_seconds * flops_s / per_tok))
+    order = np.argsort(synth.bits(synth.key(w.seed_len, 7), np.arange(w.B)))
+    reqs, tot = [], 0
+    for b in order:
+        if tot + int(w.lengths[b]) > budget_tok and reqs:
+            continue
+        reqs.append(int(b))
+        tot += int(w.lengths[b])
+        if tot >= budget_tok:
+            break
+    return sorted(reqs), tot
+
+
+def oracle_arrays(w, reqs):
+    """Dense float64 inputs of the sampled requests (generated untimed)."""
+    import oracle
+    Lmax = int(max(w.lengths[b] for b in reqs))
+    B = len(reqs)
+    q = synth.bf16_bits_to_f64(synth.q_bf16(w.seed_val, w.B, w.hq, w.dk))[reqs]
+    lens = np.array([w.lengths[b] for b in reqs], np.int64)
+    if w.kind == "gqa":
+        K = np.zeros((B, Lmax, w.hkv, w.dk))
+        V = np.zeros((B, Lmax, w.hkv, w.dv))
+        for i, b in enumerate(reqs):
+            K[i, :lens[i]] = synth.bf16_bits_to_f64(synth.kv_rows_bf16(w.seed_val, synth.T_K, b, np.arange(lens[i]),
+                                                                        w.hkv, w.dk))
+            V[i, :lens[i]] = synth.bf16_bits_to_f64(synth.kv_rows_bf16(w.seed_val, synth.T_V, b, np.arange(lens[i]),
+                                                                        w.hkv, w.dv))
+        return q, K, V, lens
+    K = np.zeros((B, Lmax, 576))
+    for i, b in enumerate(reqs):
+        rows = synth.kv_rows_bf16(w.seed_val, synth.T_LATENT, b, np.arange(lens[i]), 1, 576)[:, 0]
+        if w.dtype == "fp8":
+            codes, sc = oracle.quantize_rows_e4m3(rows)
+            K[i, :lens[i]] = _E4M3[codes] * sc.astype(np.float64)[:, None]
+        else:
+            K[i, :lens[i]] = synth.bf16_bits_to_f64(rows)
+    return q, K, None, lens
+
+
+_E4M3 = None
+
+
+def _init_e4m3():
+    global _E4M3
+    import oracle
+    _E4M3 = oracle.e4m3_table()
+
+
+def time_oracle(w, cpu_seconds: float):
+    """Time the oracle (as it stands) on a bounded sample; returns dict."""
+    import oracle
+    _init_e4m3()
+    reqs, tot = oracle_sample(w, cpu_seconds)
+    q, K, V, lens = oracle_arrays(w, reqs)
+    t0 = time.perf_counter()
+    oracle.decode_arrays(w.kind, q, K, V, lens, w.scale, dv=w.dv)
+    dt = time.perf_counter() - t0
+    kv_bytes = int(lens.sum()) * w.kv_bytes_per_token
+    return {"value": round(kv_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+            "sample": f"{len(reqs)} of {w.B} requests ({int(lens.sum())} tokens, all {w.hq} heads, unsharded "
+                      f"float64 decode attention), {dt:.1f} s"}, dt, kv_bytes
+
+
+def run_reference(args):
+    w = get_workload(args)
+    per_step = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
+    import oracle
+    _init_e4m3()
+    reqs, tot = oracle_sample(w, per_step)
+    q, K, V, lens = oracle_arrays(w, reqs)
+    kv_bytes = int(lens.sum()) * w.kv_bytes_per_token
+    for _ in range(args.warmup):
+        oracle.decode_arrays(w.kind, q, K, V, lens, w.scale, dv=w.dv)
+    t0 = time.perf_counter()
+    for _ in range(args.steps):
+        oracle.decode_arrays(w.kind, q, K, V, lens, w.scale, dv=w.dv)
+    dt = time.perf_counter() - t0
+    gbs = kv_bytes * args.steps / dt / 1e9
+    sample = (f"each step: {len(reqs)} of {w.B} requests ({int(lens.sum())} tokens, all {w.hq} heads) "
+              f"of the workload, unsharded float64 decode attention on host cores")
+    return {
+        "impl": "reference",
+        "metric": METRIC, "value": round(gbs, 4), "unit": "GB/s", "n_gpus": 1,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+        "data": "synthetic (seeded counter-based generator)",
+        "config": workload_config(w, args) | {"parallelism": "host cores (OpenMP)"},
+        "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
+                         "sample": sample},
+        "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse()
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if args.impl == "reference":
+        if rank == 0:
+            print(json.dumps(run_reference(args)), flush=True)
+        return
+    import torch
+    import torch.distributed as dist
+    if world > 1:
+        import datetime
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        res, w = run_ours(args, rank, world, local_rank)
+        if rank == 0 and not args.no_cpu_baseline:
+            cb, _, _ = time_oracle(w, args.cpu_seconds)
+            res["cpu_baseline"] = cb
+        if rank == 0:
+            print(json.dumps(res), flush=True)
+    finally:
+        if world > 1:
+            dist.barrier()
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

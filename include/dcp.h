@@ -1,0 +1,214 @@
+/*
+ * dcp.h -- C ABI of libdcp: decode attention over a paged KV cache that is
+ * sharded along the sequence (Decode Context Parallelism), for NVIDIA B200
+ * (sm_100a).
+ *
+ * The method (web pages on Decode Context Parallelism):
+ *  - "Efficient Decode Context Parallelism with vLLM for Long Context
+ *    Workloads", section 4: every GPU of the group keeps the KV cache of a
+ *    subset of the token positions of each request, so per-GPU KV is 1/N;
+ *  - same page, section 4.1: each GPU attends the (gathered) query against its
+ *    local KV slice, producing a partial output and a per-head log-sum-exp;
+ *    the partials are reweighted by their LSE and summed (all-gather +
+ *    reduce-scatter across GPUs);
+ *  - same page, sections 5.3 / 5.4: MLA keeps one latent row per token shared
+ *    by all query heads; GQA broadcasts each KV head to its query heads;
+ *  - "Decode Context Parallel Guide" (vLLM Ascend), Constraints:
+ *    cp_kv_cache_interleave_size sets how many consecutive positions go to
+ *    one shard before moving to the next.
+ *
+ * This library runs all N shards on ONE GPU: shard n's pages live in the same
+ * page pool as the other shards' pages (disjoint page ids), decode_partial
+ * computes every shard's partial in one launch, and dcp_merge performs the
+ * LSE-weighted sum that the all-gather + reduce-scatter would perform across
+ * GPUs.
+ *
+ * Conventions for every call:
+ *  - Every pointer argument is DEVICE memory owned by the caller, unless the
+ *    argument's comment says "host".  The library allocates nothing and keeps
+ *    no pointer after a call returns.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Work is
+ *    enqueued asynchronously; the return value reports host-side validation
+ *    and launch errors only.  Errors found by a kernel (an unallocated page,
+ *    a negative length) are recorded in a sticky per-device status word read
+ *    by dcp_get_device_status(); kernels never trap and never spin without a
+ *    time limit.
+ *  - Device pointers must be 16-byte aligned (DCP_ERR_MISALIGNED otherwise).
+ *  - Sizes are element counts unless they say bytes.
+ */
+#ifndef DCP_H
+#define DCP_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+    DCP_OK = 0,
+    DCP_ERR_INVALID_ARG = 1,        /* a size, count or pointer is out of range / NULL */
+    DCP_ERR_UNSUPPORTED = 2,        /* a valid shape this build has no kernel for */
+    DCP_ERR_UNALLOCATED_PAGE = 3,   /* a block-table entry needed by the call is not a pool page */
+    DCP_ERR_WORKSPACE_TOO_SMALL = 4,
+    DCP_ERR_CUDA = 5,               /* a CUDA runtime call failed (launch, attribute, ...) */
+    DCP_ERR_MISALIGNED = 6,         /* a device pointer is not 16-byte aligned */
+    DCP_ERR_TIMEOUT = 7             /* a kernel gave up waiting on a copy (never expected) */
+} dcp_status;
+
+typedef enum { DCP_GQA = 0, DCP_MLA = 1 } dcp_kind;
+typedef enum { DCP_BF16 = 0, DCP_FP8_E4M3 = 1 } dcp_dtype;
+
+/*
+ * The sharded paged KV cache.
+ *
+ *  kind/dtype   DCP_GQA with DCP_BF16; or DCP_MLA with DCP_BF16 or DCP_FP8_E4M3.
+ *  n_shards     N >= 1: shards of the sequence dimension.
+ *  interleave   I >= 1: position p belongs to shard (p / I) mod N; within a
+ *               shard the owned positions are packed in increasing order, so
+ *               p has local index (p / (I*N))*I + p mod I.
+ *  page_size    P tokens per page: 16 or 64.
+ *  num_pages    pages in the pool (all shards together).
+ *  hq, hkv      query heads and KV heads (MLA: hkv = 1); hq % hkv == 0; query
+ *               head h reads KV head h / (hq/hkv).
+ *  dk, dv       key and value widths.  GQA: dk = dv in {64, 128}.  MLA: dk =
+ *               576 (512 + 64 rope), dv = 512; the value is the first dv
+ *               entries of the latent row (absorbed MLA).
+ *  scale        softmax scale applied to q.k.
+ *  k_pages      GQA: keys   [num_pages][hkv][P][dk] bf16.
+ *               MLA: latent [num_pages][P][576] bf16, or e4m3 bytes for fp8.
+ *  v_pages      GQA: values [num_pages][hkv][P][dv] bf16.  MLA: NULL.
+ *  kv_scales    MLA fp8: per-token fp32 scale [num_pages][P]; value of latent
+ *               element = e4m3(code) * scale.  Otherwise NULL.
+ *  block_tables int32 [n_shards][batch][max_local_pages]: shard n's local page
+ *               j of request b is pool page block_tables[n][b][j]; -1 = none.
+ *  batch        B: requests (rows of each shard's block table).
+ */
+typedef struct {
+    int32_t kind;
+    int32_t dtype;
+    int32_t n_shards;
+    int32_t interleave;
+    int32_t page_size;
+    int32_t num_pages;
+    int32_t hq;
+    int32_t hkv;
+    int32_t dk;
+    int32_t dv;
+    float scale;
+    int32_t batch;
+    int32_t max_local_pages;
+    int32_t reserved0;
+    void* k_pages;
+    void* v_pages;
+    float* kv_scales;
+    const int32_t* block_tables;
+} dcp_cache_desc;
+
+/* Human-readable name of a status code (static string, host). */
+const char* dcp_status_string(dcp_status s);
+
+/*
+ * dcp_shard_counts -- positions each shard owns.
+ * Passage: blog section 4 (positions split across GPUs) and the guide's
+ * cp_kv_cache_interleave_size.
+ *  seq_lens   int32 [B]: logical lengths L_b >= 0.
+ *  counts_out int32 [N][B]: number of p in [0, L_b) with (p / I) mod N == n,
+ *             i.e. (L/(I N))*I + clamp(L mod (I N) - n I, 0, I).
+ * Errors: DCP_ERR_INVALID_ARG for B < 1, N < 1, I < 1 or NULL pointers.
+ */
+dcp_status dcp_shard_counts(int32_t B, const int32_t* seq_lens, int32_t N, int32_t I, int32_t* counts_out,
+                            void* stream);
+
+/*
+ * dcp_shard_map -- owner and storage slot of positions.
+ * Passage: blog section 4; the guide's cp_kv_cache_interleave_size.
+ *  n_pos      number of positions.
+ *  pos        int32 [n_pos]: positions p >= 0.
+ *  req        int32 [n_pos]: request of each position, or NULL (position i
+ *             belongs to request i).
+ *  rank_out   int32 [n_pos]: owner shard (p / I) mod N.
+ *  local_out  int32 [n_pos]: local index (p / (I N))*I + p mod I.
+ *  slot_out   int64 [n_pos]: physical slot block_tables[rank][req][local / P] * P
+ *             + local mod P, or -1 when that block-table entry is -1 or not a
+ *             pool page (the device status word then records
+ *             DCP_ERR_UNALLOCATED_PAGE).
+ * Uses n_shards, interleave, page_size, num_pages, batch, max_local_pages and
+ * block_tables of `cache` (page pools may be NULL).
+ */
+dcp_status dcp_shard_map(const dcp_cache_desc* cache, int64_t n_pos, const int32_t* pos, const int32_t* req,
+                         int32_t* rank_out, int32_t* local_out, int64_t* slot_out, void* stream);
+
+/*
+ * dcp_kv_append -- write tokens into the pages of the shard that owns them.
+ * Passage: blog section 4 (a position's KV lives only on its owner) and
+ * sections 5.3 / 5.4 (latent row vs. per-KV-head rows).
+ *  n_tok      rows to write (one decode step: n_tok = B, pos = L_b).
+ *  req        int32 [n_tok] request of each row, or NULL (row i -> request i).
+ *  pos        int32 [n_tok] position of each row.
+ *  k_new      GQA: bf16 [n_tok][hkv][dk].  MLA: latent bf16 [n_tok][576]; for an
+ *             fp8 cache the row is quantised on the way in: scale = amax/448
+ *             (fp32), code = round-to-nearest-even(x / scale) saturated to
+ *             +-448; amax = 0 stores scale 1 and zero codes.
+ *  v_new      GQA: bf16 [n_tok][hkv][dv].  MLA: NULL.
+ * Rows whose slot is unallocated are skipped and the device status word
+ * records DCP_ERR_UNALLOCATED_PAGE.  Two rows with the same (req, pos) race.
+ */
+dcp_status dcp_kv_append(const dcp_cache_desc* cache, int64_t n_tok, const int32_t* req, const int32_t* pos,
+                         const void* k_new, const void* v_new, void* stream);
+
+/*
+ * dcp_decode_workspace_size -- bytes of device workspace dcp_decode_partial
+ * needs for this cache and batch on the CURRENT device (host function; no
+ * GPU work).  Returns 0 for an invalid descriptor.
+ */
+size_t dcp_decode_workspace_size(const dcp_cache_desc* cache, int32_t B);
+
+/*
+ * dcp_decode_partial -- every shard's partial decode attention, one launch
+ * sequence for all N shards.
+ * Passage: blog section 4.1 ("Compute": attention between the gathered query
+ * and the local KV slice, giving a partial output and its LSE).
+ *  B          requests; must equal cache->batch.
+ *  q          bf16 [B][hq][dk]: one query token per request (already
+ *             gathered; on one GPU every shard reads the same q).
+ *  seq_lens   int32 [B]: L_b, positions [0, L_b) are attended.
+ *  o_partial  fp32 [N][B][hq][dv]: shard n's normalised partial output
+ *             sum_p exp(s_p - m) v_p / sum_p exp(s_p - m) over its own
+ *             positions, s_p = scale * q . k_p; 0 when shard n owns none.
+ *  lse        fp32 [N][B][hq]: natural-log LSE of shard n's scores,
+ *             -inf when it owns none.
+ *  ws, ws_bytes  device workspace of at least dcp_decode_workspace_size()
+ *             bytes; its contents need no initialisation and are clobbered.
+ * Concurrent calls must use distinct workspaces.
+ */
+dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void* q, const int32_t* seq_lens,
+                              float* o_partial, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * dcp_merge -- LSE-weighted merge of N partials (the arithmetic of the
+ * all-gather + reduce-scatter step).
+ * Passage: blog section 4.1 ("the LSE values reweight and merge the partials").
+ *  o_partial  fp32 [N][B][H][Dv], lse fp32 [N][B][H] (as written by
+ *             dcp_decode_partial).
+ *  out        fp32 [B][H][Dv]: sum_n exp(lse_n - LSE) o_n.
+ *  lse_out    fp32 [B][H]: LSE = M + ln sum_n exp(lse_n - M), M = max_n lse_n;
+ *             all -inf gives out = 0, LSE = -inf.  May be NULL.
+ */
+dcp_status dcp_merge(int32_t N, int32_t B, int32_t H, int32_t Dv, const float* o_partial, const float* lse,
+                     float* out, float* lse_out, void* stream);
+
+/*
+ * dcp_get_device_status -- read and clear the sticky device status word of
+ * the current device.  Synchronises `stream` first.
+ *  status_out  HOST int32: DCP_OK, or the first error a kernel recorded since
+ *              the last read.
+ */
+dcp_status dcp_get_device_status(int32_t* status_out, void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* DCP_H */

@@ -88,6 +88,8 @@ def lib():
         L.orc_e4m3_encode.restype = ctypes.c_uint8
         L.orc_quantize_row_e4m3.argtypes = [P, ctypes.c_int32, P, P]
         L.orc_quantize_row_e4m3.restype = None
+        L.orc_quantize_rows_e4m3.argtypes = [ctypes.c_int64, ctypes.c_int32, P, P, P]
+        L.orc_quantize_rows_e4m3.restype = None
         L.orc_decode.argtypes = [ctypes.POINTER(_Cache), P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                  P, ctypes.c_int32, P, P]
         L.orc_decode.restype = ctypes.c_int
@@ -161,6 +163,21 @@ def quantize_row_e4m3(row_bf16: np.ndarray):
     sc = np.zeros(1, np.float32)
     lib().orc_quantize_row_e4m3(_p(r), r.size, _p(codes), _p(sc))
     return codes, float(sc[0])
+
+
+def quantize_rows_e4m3(rows_bf16: np.ndarray):
+    """Row-wise quantisation of rows [n][W] (bf16 bits): (codes uint8 [n][W], scales float32 [n])."""
+    r = np.ascontiguousarray(rows_bf16, dtype=np.uint16)
+    n, W = r.shape
+    codes = np.zeros((n, W), np.uint8)
+    sc = np.zeros(n, np.float32)
+    lib().orc_quantize_rows_e4m3(n, W, _p(r), _p(codes), _p(sc))
+    return codes, sc
+
+
+def e4m3_table() -> np.ndarray:
+    """float64 value of each of the 256 e4m3 codes (NaN for the NaN codes)."""
+    return np.array([e4m3_decode(c) for c in range(256)])
 
 
 # ----------------------------------------------------------------------------

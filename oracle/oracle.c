@@ -174,6 +174,12 @@ void orc_quantize_row_e4m3(const uint16_t* row_bf16, int32_t W, uint8_t* codes, 
     *scale_out = scale;
 }
 
+/* n rows of width W: codes [n][W], scales [n] */
+void orc_quantize_rows_e4m3(int64_t n, int32_t W, const uint16_t* rows_bf16, uint8_t* codes, float* scales) {
+#pragma omp parallel for schedule(static)
+    for (int64_t i = 0; i < n; i++) orc_quantize_row_e4m3(rows_bf16 + i * W, W, codes + i * W, scales + i);
+}
+
 /* ------------------------------------------------------------------------ */
 /* decode attention                                                          */
 /* ------------------------------------------------------------------------ */

@@ -1,0 +1,292 @@
+// api.cu -- the C ABI of libdcp (include/dcp.h): host-side validation, the
+// sticky device status word, workspace sizing and kernel dispatch.
+#include <mutex>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dcp {
+
+// Sticky status word, one per device context.
+static __device__ int g_status;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+std::mutex g_mu;
+int* g_status_ptr[kMaxDevices] = {nullptr};
+int g_num_sms[kMaxDevices] = {0};
+
+dcp_status cuda_err(cudaError_t e) { return e == cudaSuccess ? DCP_OK : DCP_ERR_CUDA; }
+
+// device address of g_status and SM count of the current device
+dcp_status device_info(int** status, int* num_sms) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DCP_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_status_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return DCP_ERR_CUDA;
+        int sms = 0;
+        if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DCP_ERR_CUDA;
+        g_status_ptr[dev] = static_cast<int*>(p);
+        g_num_sms[dev] = sms;
+    }
+    if (status) *status = g_status_ptr[dev];
+    if (num_sms) *num_sms = g_num_sms[dev];
+    return DCP_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Shape/descriptor checks shared by every call that takes a cache.
+dcp_status check_desc(const dcp_cache_desc* c, bool need_pools) {
+    if (!c) return DCP_ERR_INVALID_ARG;
+    if (c->n_shards < 1 || c->interleave < 1 || c->num_pages < 1 || c->batch < 1 || c->max_local_pages < 1)
+        return DCP_ERR_INVALID_ARG;
+    if (c->page_size != 16 && c->page_size != 64) return DCP_ERR_UNSUPPORTED;
+    if ((int64_t)c->max_local_pages * c->page_size > ((int64_t)1 << 31) - 1) return DCP_ERR_INVALID_ARG;
+    if (!c->block_tables) return DCP_ERR_INVALID_ARG;
+    if (c->hq < 1 || c->hkv < 1 || c->hq % c->hkv) return DCP_ERR_INVALID_ARG;
+    if (c->kind == DCP_GQA) {
+        if (c->dtype != DCP_BF16) return DCP_ERR_UNSUPPORTED;
+        if (c->dk != c->dv || (c->dk != 64 && c->dk != 128)) return DCP_ERR_UNSUPPORTED;
+        if (need_pools && (!c->k_pages || !c->v_pages)) return DCP_ERR_INVALID_ARG;
+        if (need_pools && (!aligned16(c->k_pages) || !aligned16(c->v_pages))) return DCP_ERR_MISALIGNED;
+    } else if (c->kind == DCP_MLA) {
+        if (c->hkv != 1 || c->dk != 576 || c->dv != 512) return DCP_ERR_UNSUPPORTED;
+        if (c->hq % 16) return DCP_ERR_UNSUPPORTED;
+        if (c->dtype != DCP_BF16 && c->dtype != DCP_FP8_E4M3) return DCP_ERR_INVALID_ARG;
+        if (need_pools && !c->k_pages) return DCP_ERR_INVALID_ARG;
+        if (need_pools && c->dtype == DCP_FP8_E4M3 && !c->kv_scales) return DCP_ERR_INVALID_ARG;
+        if (need_pools && (!aligned16(c->k_pages) || (c->kv_scales && !aligned16(c->kv_scales))))
+            return DCP_ERR_MISALIGNED;
+    } else {
+        return DCP_ERR_INVALID_ARG;
+    }
+    if (!aligned16(c->block_tables)) return DCP_ERR_MISALIGNED;
+    return DCP_OK;
+}
+
+struct Plan {
+    DecodeGeometry g;
+    WsLayout lay;
+};
+
+bool make_plan(const dcp_cache_desc* c, int B, int num_sms, Plan* p) {
+    if (!decode_geometry(c->kind, c->dtype, c->hq, c->hkv, c->dk, c->dv, c->page_size, num_sms, &p->g)) return false;
+    const int64_t target = (int64_t)p->g.units_per_cta * p->g.ctas;
+    const int64_t max_units = (int64_t)c->n_shards * B + target + 1;
+    const int64_t max_split = 2 * target + 2;
+    if (max_units > (1 << 30)) return false;
+    p->lay = ws_layout(c->n_shards, B, c->hq, c->dv, (int)max_units, (int)max_split);
+    return true;
+}
+
+}  // namespace
+
+// ---------------------------------------------------------------------------
+// decode dispatch
+// ---------------------------------------------------------------------------
+bool decode_geometry(int kind, int dtype, int hq, int hkv, int dk, int dv, int page_size, int num_sms,
+                     DecodeGeometry* g) {
+    (void)dv;
+    if (kind == DCP_GQA) {
+        const int G = hq / hkv;
+        if (G != 1 && G != 2 && G != 4 && G != 8) return false;
+        const int occ = simt_blocks_per_sm(DecodePath::GqaSimt, dk, G, page_size, false);
+        if (occ < 1) return false;
+        g->path = DecodePath::GqaSimt;
+        g->n_hb = hkv;
+        g->ctas = num_sms * occ;
+        g->granule = page_size;
+        g->min_chunk = 512;
+        g->units_per_cta = 4;
+        return true;
+    }
+    if (kind == DCP_MLA) {
+        const int occ = simt_blocks_per_sm(DecodePath::MlaSimt, dk, hq, page_size, dtype == DCP_FP8_E4M3);
+        if (occ < 1) return false;
+        g->path = DecodePath::MlaSimt;
+        g->n_hb = hq / 16;
+        g->ctas = num_sms * occ;
+        g->granule = page_size;
+        g->min_chunk = 1024;
+        g->units_per_cta = 4;
+        return true;
+    }
+    return false;
+}
+
+cudaError_t launch_decode(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s) {
+    switch (g.path) {
+        case DecodePath::GqaSimt:
+        case DecodePath::MlaSimt:
+            return launch_decode_simt(g, a, s);
+        default:
+            return cudaErrorNotSupported;
+    }
+}
+
+}  // namespace dcp
+
+using namespace dcp;
+
+extern "C" {
+
+const char* dcp_status_string(dcp_status s) {
+    switch (s) {
+        case DCP_OK: return "ok";
+        case DCP_ERR_INVALID_ARG: return "invalid argument";
+        case DCP_ERR_UNSUPPORTED: return "unsupported shape";
+        case DCP_ERR_UNALLOCATED_PAGE: return "unallocated page";
+        case DCP_ERR_WORKSPACE_TOO_SMALL: return "workspace too small";
+        case DCP_ERR_CUDA: return "CUDA error";
+        case DCP_ERR_MISALIGNED: return "misaligned pointer";
+        case DCP_ERR_TIMEOUT: return "kernel wait timed out";
+    }
+    return "unknown status";
+}
+
+dcp_status dcp_shard_counts(int32_t B, const int32_t* seq_lens, int32_t N, int32_t I, int32_t* counts_out,
+                            void* stream) {
+    if (B < 1 || N < 1 || I < 1 || !seq_lens || !counts_out) return DCP_ERR_INVALID_ARG;
+    int* status = nullptr;
+    dcp_status st = device_info(&status, nullptr);
+    if (st != DCP_OK) return st;
+    return cuda_err(launch_shard_counts(B, seq_lens, N, I, counts_out, status, (cudaStream_t)stream));
+}
+
+dcp_status dcp_shard_map(const dcp_cache_desc* cache, int64_t n_pos, const int32_t* pos, const int32_t* req,
+                         int32_t* rank_out, int32_t* local_out, int64_t* slot_out, void* stream) {
+    dcp_status st = check_desc(cache, false);
+    if (st != DCP_OK) return st;
+    if (n_pos < 0) return DCP_ERR_INVALID_ARG;
+    if (n_pos == 0) return DCP_OK;
+    if (!pos || !rank_out || !local_out || !slot_out) return DCP_ERR_INVALID_ARG;
+    int* status = nullptr;
+    st = device_info(&status, nullptr);
+    if (st != DCP_OK) return st;
+    return cuda_err(launch_shard_map(n_pos, pos, req, cache->n_shards, cache->interleave, cache->page_size,
+                                     cache->block_tables, cache->batch, cache->max_local_pages, cache->num_pages,
+                                     rank_out, local_out, slot_out, status, (cudaStream_t)stream));
+}
+
+dcp_status dcp_kv_append(const dcp_cache_desc* cache, int64_t n_tok, const int32_t* req, const int32_t* pos,
+                         const void* k_new, const void* v_new, void* stream) {
+    dcp_status st = check_desc(cache, true);
+    if (st != DCP_OK) return st;
+    if (n_tok < 0) return DCP_ERR_INVALID_ARG;
+    if (n_tok == 0) return DCP_OK;
+    if (!pos || !k_new || (cache->kind == DCP_GQA && !v_new)) return DCP_ERR_INVALID_ARG;
+    if (!aligned16(k_new) || (v_new && !aligned16(v_new))) return DCP_ERR_MISALIGNED;
+    int* status = nullptr;
+    st = device_info(&status, nullptr);
+    if (st != DCP_OK) return st;
+    AppendArgs a;
+    a.kind = cache->kind;
+    a.dtype = cache->dtype;
+    a.n_shards = cache->n_shards;
+    a.interleave = cache->interleave;
+    a.page_size = cache->page_size;
+    a.num_pages = cache->num_pages;
+    a.batch = cache->batch;
+    a.max_local_pages = cache->max_local_pages;
+    a.hkv = cache->hkv;
+    a.dk = cache->dk;
+    a.dv = cache->dv;
+    a.n_tok = n_tok;
+    a.req = req;
+    a.pos = pos;
+    a.k_new = static_cast<const uint8_t*>(k_new);
+    a.v_new = static_cast<const uint8_t*>(v_new);
+    a.k_pages = static_cast<uint8_t*>(cache->k_pages);
+    a.v_pages = static_cast<uint8_t*>(cache->v_pages);
+    a.kv_scales = cache->kv_scales;
+    a.block_tables = cache->block_tables;
+    a.status = status;
+    return cuda_err(launch_append(a, (cudaStream_t)stream));
+}
+
+size_t dcp_decode_workspace_size(const dcp_cache_desc* cache, int32_t B) {
+    if (check_desc(cache, false) != DCP_OK || B != cache->batch) return 0;
+    int num_sms = 0;
+    if (device_info(nullptr, &num_sms) != DCP_OK) return 0;
+    Plan p;
+    if (!make_plan(cache, B, num_sms, &p)) return 0;
+    return p.lay.total;
+}
+
+dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void* q, const int32_t* seq_lens,
+                              float* o_partial, float* lse, void* ws, size_t ws_bytes, void* stream) {
+    dcp_status st = check_desc(cache, true);
+    if (st != DCP_OK) return st;
+    if (B != cache->batch || !q || !seq_lens || !o_partial || !lse || !ws) return DCP_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(o_partial) || !aligned16(lse) || !aligned16(ws)) return DCP_ERR_MISALIGNED;
+    int* status = nullptr;
+    int num_sms = 0;
+    st = device_info(&status, &num_sms);
+    if (st != DCP_OK) return st;
+    Plan p;
+    if (!make_plan(cache, B, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
+    if (ws_bytes < p.lay.total) return DCP_ERR_WORKSPACE_TOO_SMALL;
+    cudaStream_t s = (cudaStream_t)stream;
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    const int64_t target = (int64_t)p.g.units_per_cta * p.g.ctas;
+    cudaError_t e = launch_plan(seq_lens, B, cache->n_shards, cache->interleave, p.g.granule, p.g.min_chunk,
+                                (int)target, p.g.n_hb, ws, p.lay.max_units, p.lay.max_split, cache->hq, cache->dv,
+                                status, s);
+    if (e != cudaSuccess) return DCP_ERR_CUDA;
+    DecodeArgs a;
+    a.k_pages = static_cast<const uint8_t*>(cache->k_pages);
+    a.v_pages = static_cast<const uint8_t*>(cache->v_pages);
+    a.kv_scales = cache->dtype == DCP_FP8_E4M3 ? cache->kv_scales : nullptr;
+    a.block_tables = cache->block_tables;
+    a.n_shards = cache->n_shards;
+    a.interleave = cache->interleave;
+    a.page_size = cache->page_size;
+    a.num_pages = cache->num_pages;
+    a.batch = B;
+    a.max_local_pages = cache->max_local_pages;
+    a.hq = cache->hq;
+    a.hkv = cache->hkv;
+    a.dk = cache->dk;
+    a.dv = cache->dv;
+    a.scale_log2 = cache->scale * kLog2e;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.seq_lens = seq_lens;
+    a.o_partial = o_partial;
+    a.lse = lse;
+    a.plan = reinterpret_cast<const PlanHeader*>(w);
+    a.units = reinterpret_cast<const Unit*>(w + p.lay.off_units);
+    a.done = reinterpret_cast<int32_t*>(w + p.lay.off_done);
+    a.split_o = reinterpret_cast<float*>(w + p.lay.off_split_o);
+    a.split_lse = reinterpret_cast<float*>(w + p.lay.off_split_lse);
+    a.status = status;
+    e = launch_decode(p.g, a, s);
+    if (e == cudaErrorNotSupported) return DCP_ERR_UNSUPPORTED;
+    return cuda_err(e);
+}
+
+dcp_status dcp_merge(int32_t N, int32_t B, int32_t H, int32_t Dv, const float* o_partial, const float* lse,
+                     float* out, float* lse_out, void* stream) {
+    if (N < 1 || B < 1 || H < 1 || Dv < 4 || Dv % 4 || !o_partial || !lse || !out) return DCP_ERR_INVALID_ARG;
+    if (!aligned16(o_partial) || !aligned16(out)) return DCP_ERR_MISALIGNED;
+    return cuda_err(launch_merge(N, B, H, Dv, o_partial, lse, out, lse_out, (cudaStream_t)stream));
+}
+
+dcp_status dcp_get_device_status(int32_t* status_out, void* stream) {
+    if (!status_out) return DCP_ERR_INVALID_ARG;
+    int* status = nullptr;
+    dcp_status st = device_info(&status, nullptr);
+    if (st != DCP_OK) return st;
+    cudaStream_t s = (cudaStream_t)stream;
+    if (cudaStreamSynchronize(s) != cudaSuccess) return DCP_ERR_CUDA;
+    int v = 0;
+    if (cudaMemcpy(&v, status, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return DCP_ERR_CUDA;
+    if (cudaMemset(status, 0, sizeof(int)) != cudaSuccess) return DCP_ERR_CUDA;
+    *status_out = v;
+    return DCP_OK;
+}
+
+}  // extern "C"

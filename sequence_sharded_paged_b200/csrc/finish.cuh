@@ -1,0 +1,84 @@
+// finish.cuh -- end of one work unit: store a shard's partial, or a chunk's
+// split partial and, in the last chunk of the shard to finish, the LSE merge
+// of the chunks (split-KV reduce).  The merge is the arithmetic of
+// "Efficient Decode Context Parallelism with vLLM for Long Context Workloads",
+// section 4.1 (LSE-reweighted sum of partials), applied within one shard.
+#pragma once
+
+#include "common.cuh"
+
+namespace dcp {
+
+__device__ __forceinline__ void named_barrier_sync(int id, int threads) {
+    asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
+}
+
+// Executed by the NT threads of barrier `bar_id` (tid in [0, NT)).
+//  sO   [nh][dv] normalised output of this unit for heads h0..h0+nh-1 (smem)
+//  sLse [nh]     natural-log LSE (-inf when the unit saw no token)
+//  hb / n_hb     head block of this unit and head blocks per unit (split counters
+//                are per (shard, head block))
+template <int NT>
+__device__ void finish_unit(const DecodeArgs& a, const Unit& u, int hb, int n_hb, int h0, int nh,
+                            const float* sO, const float* sLse, int* s_flag, int tid, int bar_id) {
+    const int dv = a.dv;
+    const int64_t shard = (int64_t)u.n * a.batch + u.b;
+    const int nvec = nh * dv / 4;
+    if (u.n_chunks == 1) {
+        float4* dst = reinterpret_cast<float4*>(a.o_partial + (shard * a.hq + h0) * dv);
+        const float4* src = reinterpret_cast<const float4*>(sO);
+        for (int i = tid; i < nvec; i += NT) dst[i] = src[i];
+        for (int i = tid; i < nh; i += NT) a.lse[shard * a.hq + h0 + i] = sLse[i];
+        return;
+    }
+    {
+        float4* dst = reinterpret_cast<float4*>(a.split_o + ((int64_t)u.slot * a.hq + h0) * dv);
+        const float4* src = reinterpret_cast<const float4*>(sO);
+        for (int i = tid; i < nvec; i += NT) __stcg(dst + i, src[i]);
+        for (int i = tid; i < nh; i += NT) __stcg(a.split_lse + (int64_t)u.slot * a.hq + h0 + i, sLse[i]);
+    }
+    __threadfence();
+    named_barrier_sync(bar_id, NT);
+    if (tid == 0) {
+        int old = atomicAdd(a.done + shard * n_hb + hb, 1);
+        *s_flag = (old == u.n_chunks - 1) ? 1 : 0;
+    }
+    named_barrier_sync(bar_id, NT);
+    const int last = *(volatile int*)s_flag;
+    named_barrier_sync(bar_id, NT);
+    if (!last) return;
+    __threadfence();
+    const int K = u.n_chunks;
+    for (int i = tid; i < nh * (dv / 4); i += NT) {
+        int h = i / (dv / 4), d4 = i - h * (dv / 4);
+        const float* lse_col = a.split_lse + (int64_t)u.slot_base * a.hq + h0 + h;
+        float M = -INFINITY;
+        for (int j = 0; j < K; j++) M = fmaxf(M, __ldcg(lse_col + (int64_t)j * a.hq));
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        float wsum = 0.f;
+        if (M != -INFINITY) {
+            for (int j = 0; j < K; j++) {
+                float lj = __ldcg(lse_col + (int64_t)j * a.hq);
+                if (lj == -INFINITY) continue;
+                float w = expf(lj - M);
+                wsum += w;
+                float4 x = __ldcg(reinterpret_cast<const float4*>(
+                                      a.split_o + ((int64_t)(u.slot_base + j) * a.hq + h0 + h) * dv) +
+                                  d4);
+                o.x += w * x.x;
+                o.y += w * x.y;
+                o.z += w * x.z;
+                o.w += w * x.w;
+            }
+            float inv = 1.f / wsum;
+            o.x *= inv;
+            o.y *= inv;
+            o.z *= inv;
+            o.w *= inv;
+        }
+        reinterpret_cast<float4*>(a.o_partial + (shard * a.hq + h0 + h) * dv)[d4] = o;
+        if (d4 == 0) a.lse[shard * a.hq + h0 + h] = (M == -INFINITY) ? -INFINITY : M + logf(wsum);
+    }
+}
+
+}  // namespace dcp

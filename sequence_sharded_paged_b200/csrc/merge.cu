@@ -1,0 +1,64 @@
+// merge.cu -- LSE-weighted merge of the N shard partials (dcp_merge).
+//
+// "Efficient Decode Context Parallelism with vLLM for Long Context Workloads",
+// section 4.1: the all-gathered LSE values reweight the partial outputs and
+// the reduce-scatter sums them.  With every shard on one GPU the same
+// arithmetic is one pass over o_partial:
+//   M = max_n lse_n,  LSE = M + ln sum_n exp(lse_n - M),
+//   out = sum_n exp(lse_n - LSE) * o_n.
+// HBM-bound: one warp per (b, h) row streams the N rows with 16-byte loads.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace dcp {
+
+namespace {
+
+constexpr int kMergeWarps = 8;
+
+__global__ void __launch_bounds__(32 * kMergeWarps)
+    merge_kernel(int N, int64_t BH, int Dv, const float* __restrict__ o_part, const float* __restrict__ lse_part,
+                 float* __restrict__ out, float* __restrict__ lse_out) {
+    const int64_t row = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= BH) return;
+    float M = -INFINITY;
+    for (int n = 0; n < N; n++) M = fmaxf(M, __ldg(lse_part + (int64_t)n * BH + row));
+    float4* o = reinterpret_cast<float4*>(out + row * Dv);
+    const int nv = Dv / 4;
+    if (M == -INFINITY) {
+        for (int v = lane; v < nv; v += 32) o[v] = make_float4(0.f, 0.f, 0.f, 0.f);
+        if (lane == 0 && lse_out) lse_out[row] = -INFINITY;
+        return;
+    }
+    float sum = 0.f;
+    for (int n = 0; n < N; n++) sum += expf(__ldg(lse_part + (int64_t)n * BH + row) - M);
+    const float L = M + logf(sum);
+    if (lane == 0 && lse_out) lse_out[row] = L;
+    for (int v = lane; v < nv; v += 32) {
+        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int n = 0; n < N; n++) {
+            const float ln = __ldg(lse_part + (int64_t)n * BH + row);
+            if (ln == -INFINITY) continue;
+            const float w = expf(ln - L);
+            const float4 x = __ldcs(reinterpret_cast<const float4*>(o_part + ((int64_t)n * BH + row) * Dv) + v);
+            acc.x = fmaf(w, x.x, acc.x);
+            acc.y = fmaf(w, x.y, acc.y);
+            acc.z = fmaf(w, x.z, acc.z);
+            acc.w = fmaf(w, x.w, acc.w);
+        }
+        o[v] = acc;
+    }
+}
+
+}  // namespace
+
+cudaError_t launch_merge(int N, int B, int H, int Dv, const float* o_partial, const float* lse, float* out,
+                         float* lse_out, cudaStream_t s) {
+    const int64_t BH = (int64_t)B * H;
+    const int64_t blocks = (BH + kMergeWarps - 1) / kMergeWarps;
+    merge_kernel<<<(unsigned)blocks, 32 * kMergeWarps, 0, s>>>(N, BH, Dv, o_partial, lse, out, lse_out);
+    return cudaGetLastError();
+}
+
+}  // namespace dcp

@@ -1,0 +1,102 @@
+"""The C-ABI libraries load on a CPU-only host, export every declared entry
+point, and reject bad arguments on the host before touching a GPU."""
+import ctypes
+import os
+import re
+import subprocess
+import tempfile
+
+import pytest
+
+import sequence_sharded_paged_b200 as dcp
+import synth
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "dcp.h")
+
+
+def _declared_functions():
+    text = open(HEADER).read()
+    text = re.sub(r"/\*.*?\*/", "", text, flags=re.S)
+    return sorted(set(re.findall(r"\b(dcp_[a-z_]+)\s*\(", text)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for n in ("dcp_shard_map", "dcp_shard_counts", "dcp_kv_append", "dcp_decode_workspace_size",
+              "dcp_decode_partial", "dcp_merge", "dcp_get_device_status", "dcp_status_string"):
+        assert n in names
+
+
+def test_libdcp_exports_every_declared_symbol():
+    out = subprocess.run(["nm", "-D", "--defined-only", dcp.LIB_PATH], capture_output=True, text=True, check=True)
+    exported = set(re.findall(r" T (\w+)", out.stdout))
+    missing = [n for n in _declared_functions() if n not in exported]
+    assert not missing, missing
+    lib = dcp.lib()
+    for n in _declared_functions():
+        assert hasattr(lib, n)
+
+
+def test_python_binding_names_match_header():
+    for n in _declared_functions():
+        if n == "dcp_status_string":
+            continue
+        assert callable(getattr(dcp, n)), n
+
+
+def test_status_strings():
+    assert dcp.status_string(dcp.DCP_OK) == "ok"
+    assert dcp.status_string(dcp.DCP_ERR_UNALLOCATED_PAGE) == "unallocated page"
+    assert dcp.status_string(99) == "unknown status"
+
+
+def test_cache_desc_layout_matches_c_struct():
+    src = r"""
+    #include <stdio.h>
+    #include <stddef.h>
+    #include "dcp.h"
+    int main(void) {
+      printf("%zu %zu %zu %zu %zu %zu %zu\n", sizeof(dcp_cache_desc), offsetof(dcp_cache_desc, scale),
+             offsetof(dcp_cache_desc, batch), offsetof(dcp_cache_desc, k_pages), offsetof(dcp_cache_desc, v_pages),
+             offsetof(dcp_cache_desc, kv_scales), offsetof(dcp_cache_desc, block_tables));
+      return 0;
+    }
+    """
+    with tempfile.TemporaryDirectory() as d:
+        c = os.path.join(d, "t.c")
+        exe = os.path.join(d, "t")
+        open(c, "w").write(src)
+        subprocess.run(["gcc", "-I", os.path.join(ROOT, "include"), c, "-o", exe], check=True)
+        vals = [int(x) for x in subprocess.run([exe], capture_output=True, text=True, check=True).stdout.split()]
+    D = dcp.CacheDesc
+    assert vals == [ctypes.sizeof(D), D.scale.offset, D.batch.offset, D.k_pages.offset, D.v_pages.offset,
+                    D.kv_scales.offset, D.block_tables.offset]
+
+
+def test_host_validation_without_gpu():
+    L = dcp.lib()
+    # invalid sizes are rejected before any CUDA call
+    assert L.dcp_shard_counts(0, None, 2, 1, None, None) == dcp.DCP_ERR_INVALID_ARG
+    assert L.dcp_merge(0, 1, 1, 4, None, None, None, None, None) == dcp.DCP_ERR_INVALID_ARG
+    assert L.dcp_kv_append(None, 1, None, None, None, None, None) == dcp.DCP_ERR_INVALID_ARG
+    assert L.dcp_shard_map(None, 1, None, None, None, None, None, None) == dcp.DCP_ERR_INVALID_ARG
+    assert L.dcp_get_device_status(None, None) == dcp.DCP_ERR_INVALID_ARG
+    d = dcp.CacheDesc()
+    assert L.dcp_decode_workspace_size(ctypes.byref(d), 1) == 0
+    d.kind, d.dtype, d.n_shards, d.interleave, d.page_size = dcp.DCP_MLA, dcp.DCP_BF16, 2, 1, 64
+    d.num_pages, d.hq, d.hkv, d.dk, d.dv, d.batch, d.max_local_pages = 10, 64, 1, 576, 512, 1, 4
+    d.block_tables = 16
+    assert L.dcp_decode_partial(ctypes.byref(d), 1, None, None, None, None, None, 0, None) == \
+        dcp.DCP_ERR_INVALID_ARG
+    d.page_size = 32
+    assert L.dcp_shard_map(ctypes.byref(d), 1, 16, None, 16, 16, 16, None) == dcp.DCP_ERR_UNSUPPORTED
+    d.page_size, d.dk = 64, 128
+    assert L.dcp_shard_map(ctypes.byref(d), 1, 16, None, 16, 16, 16, None) == dcp.DCP_ERR_UNSUPPORTED
+    d.dk, d.block_tables = 576, 8
+    assert L.dcp_shard_map(ctypes.byref(d), 1, 16, None, 16, 16, 16, None) == dcp.DCP_ERR_MISALIGNED
+
+
+def test_libsynth_exports():
+    lib = synth.device_lib()
+    assert hasattr(lib, "synth_fill_flat") and hasattr(lib, "synth_fill_kv_rows")

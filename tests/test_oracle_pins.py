@@ -391,3 +391,13 @@ def test_synth_source_fp8_uses_quantised_rows():
     Os, ls = oracle.decode_synth("mla", "fp8", seed, q, L, 0.1, 1, 576, 512)
     np.testing.assert_allclose(Os, Oa, rtol=0, atol=1e-15)
     np.testing.assert_allclose(ls, la, rtol=0, atol=1e-15)
+
+
+def test_quantize_rows_matches_single_rows():
+    rng = np.random.default_rng(12)
+    rows = synth.bf16_bits_from_f64(rng.standard_normal((40, 576)) * rng.uniform(0.1, 3, (40, 1)))
+    rows[3] = 0
+    codes, sc = oracle.quantize_rows_e4m3(rows)
+    for i in range(40):
+        c1, s1 = oracle.quantize_row_e4m3(rows[i])
+        assert np.array_equal(codes[i], c1) and sc[i] == np.float32(s1)
