@@ -91,6 +91,17 @@ bool make_plan(const dcp_cache_desc* c, int B, int num_sms, Plan* p) {
 bool decode_geometry(int kind, int dtype, int hq, int hkv, int dk, int dv, int page_size, int num_sms,
                      DecodeGeometry* g) {
     (void)dv;
+    if (kind == DCP_GQA && gqa_mma_supported(hq, hkv, dk)) {
+        const int occ = gqa_mma_blocks_per_sm(hq, hkv, dk);
+        if (occ < 1) return false;
+        g->path = DecodePath::GqaMma;
+        g->n_hb = 1;
+        g->ctas = num_sms * occ;
+        g->granule = page_size;
+        g->min_chunk = 1024;
+        g->units_per_cta = 4;
+        return true;
+    }
     if (kind == DCP_GQA) {
         const int G = hq / hkv;
         if (G != 1 && G != 2 && G != 4 && G != 8) return false;
@@ -123,6 +134,8 @@ cudaError_t launch_decode(const DecodeGeometry& g, const DecodeArgs& a, cudaStre
         case DecodePath::GqaSimt:
         case DecodePath::MlaSimt:
             return launch_decode_simt(g, a, s);
+        case DecodePath::GqaMma:
+            return launch_decode_gqa_mma(g, a, s);
         default:
             return cudaErrorNotSupported;
     }

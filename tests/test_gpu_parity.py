@@ -250,3 +250,18 @@ def test_invalid_arguments_raise():
     with pytest.raises(dcp.DcpError) as e:
         dcp.dcp_merge(o, lse, torch.empty((1, 8, 64), device="cuda")[:, :, 1:], None)
     assert e.value.status in (dcp.DCP_ERR_MISALIGNED, dcp.DCP_ERR_INVALID_ARG)
+
+
+# ----------------------------------------------------------------------------
+# GQA with a 16-head group: the tensor-core kernel
+# ----------------------------------------------------------------------------
+
+@pytest.mark.parametrize("hkv,D,N,I", [(4, 128, 8, 128), (4, 128, 3, 16), (1, 128, 2, 1), (2, 64, 4, 5),
+                                       (8, 128, 2, 16), (4, 64, 1, 1)])
+def test_decode_gqa_group16_tensor_core(hkv, D, N, I):
+    L = [1, 15, 16, 17, 129, 2047, 5000, 333]
+    _check_decode(small_workload("gqa", "bf16", L, 16 * hkv, hkv, D, D, 16, N, I))
+
+
+def test_decode_gqa_group16_page64():
+    _check_decode(small_workload("gqa", "bf16", [70, 64, 1000, 3], 64, 4, 128, 128, 64, 2, 64))
