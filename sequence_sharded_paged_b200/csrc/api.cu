@@ -99,7 +99,7 @@ bool decode_geometry(int kind, int dtype, int hq, int hkv, int dk, int dv, int p
         g->ctas = num_sms * occ;
         g->granule = page_size;
         g->min_chunk = 1024;
-        g->units_per_cta = 4;
+        g->units_per_cta = 16;
         return true;
     }
     if (kind == DCP_GQA) {
@@ -113,6 +113,15 @@ bool decode_geometry(int kind, int dtype, int hq, int hkv, int dk, int dv, int p
         g->granule = page_size;
         g->min_chunk = 512;
         g->units_per_cta = 4;
+        return true;
+    }
+    if (kind == DCP_MLA && mla_umma_supported(hq, page_size)) {
+        g->path = DecodePath::MlaUmma;
+        g->n_hb = 1;
+        g->ctas = num_sms;  // one CTA per SM (shared memory and the whole TMEM)
+        g->granule = page_size;
+        g->min_chunk = 2048;
+        g->units_per_cta = 16;
         return true;
     }
     if (kind == DCP_MLA) {
@@ -136,6 +145,8 @@ cudaError_t launch_decode(const DecodeGeometry& g, const DecodeArgs& a, cudaStre
             return launch_decode_simt(g, a, s);
         case DecodePath::GqaMma:
             return launch_decode_gqa_mma(g, a, s);
+        case DecodePath::MlaUmma:
+            return launch_decode_mla_umma(g, a, s);
         default:
             return cudaErrorNotSupported;
     }
@@ -271,6 +282,7 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
     a.o_partial = o_partial;
     a.lse = lse;
     a.plan = reinterpret_cast<const PlanHeader*>(w);
+    a.ticket = &reinterpret_cast<PlanHeader*>(w)->next_unit;
     a.units = reinterpret_cast<const Unit*>(w + p.lay.off_units);
     a.done = reinterpret_cast<int32_t*>(w + p.lay.off_done);
     a.split_o = reinterpret_cast<float*>(w + p.lay.off_split_o);

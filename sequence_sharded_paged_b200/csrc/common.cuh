@@ -162,8 +162,26 @@ struct PlanHeader {
     int32_t max_units;
     int32_t max_split;
     int64_t total_tokens;
-    int32_t pad[2];
+    int32_t next_unit;  // dynamic-scheduling ticket (zeroed by the planner)
+    int32_t pad;
 };
+
+// Per-stage metadata of the dynamically scheduled kernels: which unit and
+// token a ring stage holds.  Written by the producer before it arrives on the
+// stage's full barrier.
+struct StageMeta {
+    int32_t unit;   // unit index, -1 = no more work
+    int32_t t;      // first local token of the stage
+    int32_t flags;  // kStageFirst | kStageLast | kStageValid
+    int32_t sidx;   // stage index within the unit
+};
+__device__ __forceinline__ StageMeta load_meta(const StageMeta* m) {
+    const volatile int32_t* v = reinterpret_cast<const volatile int32_t*>(m);
+    return StageMeta{v[0], v[1], v[2], v[3]};
+}
+constexpr int kStageFirst = 1;
+constexpr int kStageLast = 2;
+constexpr int kStageValid = 4;
 
 // Workspace layout (all offsets 256-byte aligned):
 //   PlanHeader | Unit[max_units] | int32 done[N*B] | int32 shard_k[N*B] |
@@ -213,6 +231,7 @@ struct DecodeArgs {
     float* lse;
     // workspace
     const PlanHeader* plan;
+    int32_t* ticket;  // &plan->next_unit
     const Unit* units;
     int32_t* done;
     float* split_o;

@@ -78,6 +78,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
     float* sLse = sL + NCW * 16;                                                 // [hq]
     uint64_t* full = reinterpret_cast<uint64_t*>(sLse + a.hq + (a.hq & 1));
     uint64_t* empty = full + stages;
+    StageMeta* smeta = reinterpret_cast<StageMeta*>(empty + stages);
     __shared__ int s_flag;
     __shared__ volatile int s_abort;
 
@@ -102,35 +103,60 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
         const uint64_t pol = l2_policy_evict_first();
         int stage = 0, issued = 0;
         uint32_t phase = 0;
-        for (int ui = blockIdx.x; ui < num_units && !s_abort; ui += gridDim.x) {
-            const Unit u = a.units[ui];
-            for (int t = u.t0; t < u.t1; t += kTok) {
-                if (!mbar_wait(empty + stage, phase ^ 1, &s_abort, a.status)) break;
-                const int j = t / P, sub = (t % P) / kTok;
-                const int pg = page_of(a, u.n, u.b, j);
-                if (pg >= 0) {
-                    mbar_arrive_expect_tx(full + stage, stage_bytes);
-                    uint8_t* st = ring + (size_t)stage * stage_bytes;
-                    for (int g = 0; g < hkv; g++) {
-                        const int row = (pg * hkv + g) * P + sub * kTok;
-#pragma unroll
-                        for (int h = 0; h < HALVES; h++) {
-                            tma_load_2d(st + ((size_t)(g * HALVES + h)) * kBoxBytes, &tmK, h * 64, row, full + stage,
-                                        pol);
-                            tma_load_2d(st + ((size_t)((hkv + g) * HALVES + h)) * kBoxBytes, &tmV, h * 64, row,
-                                        full + stage, pol);
-                        }
-                    }
-                } else {
-                    record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
+        while (!s_abort) {
+            const int ui = atomicAdd(a.ticket, 1);
+            if (ui >= num_units) {
+                if (mbar_wait(empty + stage, phase ^ 1, &s_abort, a.status)) {
+                    smeta[stage] = StageMeta{-1, 0, 0, 0};
                     mbar_arrive(full + stage);
+                }
+                break;
+            }
+            const Unit u = a.units[ui];
+            const int nst = (u.t1 - u.t0 + kTok - 1) / kTok;
+            int k = 0;
+            bool ok = true;
+            do {
+                if (!mbar_wait(empty + stage, phase ^ 1, &s_abort, a.status)) {
+                    ok = false;
+                    break;
+                }
+                const int t = u.t0 + k * kTok;
+                int flags = (k == 0 ? kStageFirst : 0) | (k >= nst - 1 ? kStageLast : 0);
+                if (nst == 0) {
+                    smeta[stage] = StageMeta{ui, t, flags, k};
+                    mbar_arrive(full + stage);
+                } else {
+                    const int j = t / P, sub = (t % P) / kTok;
+                    const int pg = page_of(a, u.n, u.b, j);
+                    if (pg >= 0) {
+                        smeta[stage] = StageMeta{ui, t, flags | kStageValid, k};
+                        mbar_arrive_expect_tx(full + stage, stage_bytes);
+                        uint8_t* st = ring + (size_t)stage * stage_bytes;
+                        for (int g = 0; g < hkv; g++) {
+                            const int row = (pg * hkv + g) * P + sub * kTok;
+#pragma unroll
+                            for (int h = 0; h < HALVES; h++) {
+                                tma_load_2d(st + ((size_t)(g * HALVES + h)) * kBoxBytes, &tmK, h * 64, row,
+                                            full + stage, pol);
+                                tma_load_2d(st + ((size_t)((hkv + g) * HALVES + h)) * kBoxBytes, &tmV, h * 64, row,
+                                            full + stage, pol);
+                            }
+                        }
+                    } else {
+                        record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
+                        smeta[stage] = StageMeta{ui, t, flags, k};
+                        mbar_arrive(full + stage);
+                    }
                 }
                 issued++;
                 if (++stage == stages) {
                     stage = 0;
                     phase ^= 1;
                 }
-            }
+                k++;
+            } while (k < nst);
+            if (!ok) break;
         }
         if (s_abort) {
             int n = issued < stages ? issued : stages;
@@ -151,11 +177,17 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
     const uint32_t ring_u32 = smem_u32(ring);
     int stage = 0;
     uint32_t phase = 0;
-    for (int ui = blockIdx.x; ui < num_units; ui += gridDim.x) {
-        const Unit u = a.units[ui];
-        // Q fragments (A operand), 16 heads x D
-        uint32_t qa[D / 16][4];
-        {
+    uint32_t qa[D / 16][4];
+    float o[D / 8][4];
+    float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    Unit u = a.units[0];
+    while (true) {
+        if (!mbar_wait(full + stage, phase, &s_abort, a.status)) break;
+        const StageMeta meta = load_meta(smeta + stage);
+        if (meta.unit < 0) break;
+        if (meta.flags & kStageFirst) {
+            u = a.units[meta.unit];
+            // Q fragments (A operand), 16 heads x D
             const uint32_t* q32 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)u.b * a.hq + g * 16) * D);
 #pragma unroll
             for (int kk = 0; kk < D / 16; kk++) {
@@ -164,21 +196,15 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
                 qa[kk][2] = __ldg(q32 + (qr * D + kk * 16 + 8 + 2 * qc) / 2);
                 qa[kk][3] = __ldg(q32 + ((qr + 8) * D + kk * 16 + 8 + 2 * qc) / 2);
             }
-        }
-        float o[D / 8][4];
 #pragma unroll
-        for (int i = 0; i < D / 8; i++) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
-        float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
-        bool ok = true;
-        int sidx = 0;
-        for (int t = u.t0; t < u.t1; t += kTok, sidx++) {
-            if (!mbar_wait(full + stage, phase, &s_abort, a.status)) {
-                ok = false;
-                break;
-            }
-            const int j = t / P;
-            const bool mine = (sidx % R) == r;
-            if (mine && page_of(a, u.n, u.b, j) >= 0) {
+            for (int i = 0; i < D / 8; i++) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
+            m0 = m1 = -INFINITY;
+            l0 = l1 = 0.f;
+        }
+        {
+            const int t = meta.t;
+            const bool mine = (meta.sidx % R) == r;
+            if (mine && (meta.flags & kStageValid)) {
                 const int nvalid = min(u.t1 - t, kTok);
                 const uint32_t kbase = ring_u32 + (uint32_t)stage * stage_bytes + (uint32_t)(g * HALVES) * kBoxBytes;
                 const uint32_t vbase =
@@ -259,14 +285,14 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
                     mma_bf16(o[jn + 1], pa, b2, b3);
                 }
             }
-            __syncwarp();
-            if (lane == 0) mbar_arrive(empty + stage);
-            if (++stage == stages) {
-                stage = 0;
-                phase ^= 1;
-            }
         }
-        if (!ok) break;
+        __syncwarp();
+        if (lane == 0) mbar_arrive(empty + stage);
+        if (++stage == stages) {
+            stage = 0;
+            phase ^= 1;
+        }
+        if (!(meta.flags & kStageLast)) continue;
         // row sums over the quad
         l0 += __shfl_xor_sync(0xffffffffu, l0, 1);
         l0 += __shfl_xor_sync(0xffffffffu, l0, 2);
@@ -337,14 +363,14 @@ template <int D, int NCW>
 size_t gqa_mma_smem(int hq, int hkv, int stages) {
     const size_t stage_bytes = (size_t)hkv * 2 * (D / 64) * kBoxBytes;
     return 1024 + (size_t)stages * stage_bytes + (size_t)(hq * D + 2 * NCW * 16 + hq + 2) * 4 +
-           (size_t)2 * stages * 8;
+           (size_t)2 * stages * 8 + (size_t)stages * sizeof(StageMeta);
 }
 
 template <int D, int NCW>
 int gqa_mma_stages(int hq, int hkv) {
     const size_t stage_bytes = (size_t)hkv * 2 * (D / 64) * kBoxBytes;
     const size_t fixed = gqa_mma_smem<D, NCW>(hq, hkv, 0);
-    size_t n = (200 * 1024 - fixed) / (stage_bytes + 16);
+    size_t n = (200 * 1024 - fixed) / (stage_bytes + 16 + sizeof(StageMeta));
     return (int)(n < 2 ? 2 : (n > 8 ? 8 : n));
 }
 

@@ -57,6 +57,9 @@ int simt_blocks_per_sm(DecodePath p, int D, int G, int P, bool fp8);
 bool gqa_mma_supported(int hq, int hkv, int dk);
 int gqa_mma_blocks_per_sm(int hq, int hkv, int dk);
 cudaError_t launch_decode_gqa_mma(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s);
+bool mla_umma_supported(int hq, int page_size);
+size_t mla_umma_smem_bytes(bool fp8);
+cudaError_t launch_decode_mla_umma(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s);
 
 cudaError_t launch_merge(int N, int B, int H, int Dv, const float* o_partial, const float* lse, float* out,
                          float* lse_out, cudaStream_t s);

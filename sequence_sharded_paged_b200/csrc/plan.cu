@@ -134,6 +134,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
         hdr->max_units = lay.max_units;
         hdr->max_split = lay.max_split;
         hdr->total_tokens = T;
+        hdr->next_unit = 0;
         if (!fits) record_status(status, DCP_ERR_WORKSPACE_TOO_SMALL);
     }
     if (!fits) return;

@@ -15,7 +15,7 @@ bool make_tmap_2d(CUtensorMap* map, const void* base, CUtensorMapDataType dtype,
                   uint64_t row_bytes, uint32_t box_inner, uint32_t box_outer, CUtensorMapSwizzle swizzle);
 
 #if defined(__CUDACC__)
-// 2-D tiled load (no multicast) into shared memory, completion on `bar`.
+// 2-D tiled load into this CTA's shared memory, completion on `bar`.
 // x (innermost coordinate) times the element size must be a multiple of 16 B.
 __device__ __forceinline__ void tma_load_2d(void* smem_dst, const CUtensorMap* map, int32_t x, int32_t y,
                                             uint64_t* bar, uint64_t policy) {

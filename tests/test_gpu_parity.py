@@ -265,3 +265,15 @@ def test_decode_gqa_group16_tensor_core(hkv, D, N, I):
 
 def test_decode_gqa_group16_page64():
     _check_decode(small_workload("gqa", "bf16", [70, 64, 1000, 3], 64, 4, 128, 128, 64, 2, 64))
+
+
+def test_decode_mla_page16_cuda_core_path():
+    # page size 16 is served by the CUDA-core MLA kernel
+    _check_decode(small_workload("mla", "bf16", [1, 200, 3000], 16, 1, 576, 512, 16, 2, 1))
+    _check_decode(small_workload("mla", "fp8", [17, 900], 32, 1, 576, 512, 16, 3, 4))
+
+
+@pytest.mark.parametrize("hq", [16, 32, 64])
+@pytest.mark.parametrize("dtype", ["bf16", "fp8"])
+def test_decode_mla_heads(hq, dtype):
+    _check_decode(small_workload("mla", dtype, [31, 32, 33, 64, 97, 4100], hq, 1, 576, 512, 64, 2, 1))
