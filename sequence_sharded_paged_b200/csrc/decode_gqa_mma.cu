@@ -8,8 +8,11 @@
 // Roofline: a group of 16 heads does 2*16*(D + D) = 64*D flop per token per KV
 // head for 4*D bytes of K+V, i.e. 16 flop/byte: ~105 TFLOP/s at the measured
 // 6.5 TB/s, beyond the CUDA-core fp32 rate but far below the tensor pipe, so
-// the kernel is HBM-bound and uses warp-level mma.sync m16n8k16 (bf16 in, fp32
-// accumulate): the 16 heads of a KV head fill M exactly, tokens are N.
+// the kernel is HBM-bound and uses warp-level mma.sync m16n8k16 (fp32
+// accumulate): the 16 heads of a KV head fill M exactly, tokens are N.  Q K^T
+// runs in bf16 (exact products); P V runs in f16 so that P keeps 11
+// significant bits (V fragments are widened in registers, saturating at
+// +-65504).
 //
 // Structure: persistent grid, one work unit (shard, request, chunk) per CTA
 // iteration, all KV heads in the CTA.  Warp NCW (producer) issues TMA tiled
@@ -51,9 +54,24 @@ __device__ __forceinline__ void mma_bf16(float* d, const uint32_t* a, uint32_t b
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
-    __nv_bfloat162 v = __floats2bfloat162_rn(lo, hi);
+__device__ __forceinline__ void mma_f16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
+    asm volatile(
+        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
+        "{%0, %1, %2, %3};"
+        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
+        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
+}
+
+__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
+    __half2 v = __floats2half2_rn(lo, hi);
     return *reinterpret_cast<uint32_t*>(&v);
+}
+
+// two bf16 (one 32-bit register) -> two f16, saturating at +-65504
+__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
+    const float lo = fminf(fmaxf(__uint_as_float(w << 16), -65504.f), 65504.f);
+    const float hi = fminf(fmaxf(__uint_as_float(w & 0xFFFF0000u), -65504.f), 65504.f);
+    return pack_f16(lo, hi);
 }
 
 // byte offset of (row r, column c) inside one [16][64] bf16 box with 128-byte swizzle
@@ -258,8 +276,9 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
                     o[i][2] *= c1;
                     o[i][3] *= c1;
                 }
-                uint32_t pa[4] = {pack_bf16(p[0][0], p[0][1]), pack_bf16(p[0][2], p[0][3]),
-                                  pack_bf16(p[1][0], p[1][1]), pack_bf16(p[1][2], p[1][3])};
+                // P V in f16 (11 significant bits for P): V fragments are widened in registers
+                uint32_t pa[4] = {pack_f16(p[0][0], p[0][1]), pack_f16(p[0][2], p[0][3]),
+                                  pack_f16(p[1][0], p[1][1]), pack_f16(p[1][2], p[1][3])};
                 // rows past the unit's last token hold stale page contents: zero them so that
                 // P = 0 cannot meet a NaN/Inf in the P V product
                 if (nvalid < kTok) {
@@ -281,8 +300,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
                     const uint32_t addr = vbase + (uint32_t)(col / 64) * kBoxBytes + swz(tok, col & 63);
                     uint32_t b0, b1, b2, b3;
                     ldsm_x4_t(addr, b0, b1, b2, b3);
-                    mma_bf16(o[jn], pa, b0, b1);
-                    mma_bf16(o[jn + 1], pa, b2, b3);
+                    mma_f16(o[jn], pa, bf16x2_to_f16x2(b0), bf16x2_to_f16x2(b1));
+                    mma_f16(o[jn + 1], pa, bf16x2_to_f16x2(b2), bf16x2_to_f16x2(b3));
                 }
             }
         }

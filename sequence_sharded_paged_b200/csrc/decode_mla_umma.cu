@@ -27,6 +27,9 @@
 // raw ring; four dequantising warps widen them to f16 (exact for every e4m3
 // value) into a 2-deep ring of MMA tiles, and the MMAs run as kind::f16 with
 // f16 operands.  The per-token scale multiplies the scores and P.
+// P V always runs in f16 (P has 11 significant bits instead of bf16's 8): for a
+// bf16 cache the softmax warps widen the tile's value columns to f16 in place
+// once S has consumed them (values beyond +-65504 saturate).
 //
 // Warp roles (one CTA per SM, persistent, units taken from an atomic ticket):
 //   warp 0      TMA / bulk-copy producer (lane 0)
@@ -139,7 +142,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
     constexpr int NTILE = FP8 ? kNumTilesF8 : kNumTiles16;
     constexpr uint32_t FMT = FP8 ? 0u : 1u;  // f16 : bf16
     constexpr uint32_t IDESC_S = umma::idesc_f16(FMT, 0, 0, 64, kT);
-    constexpr uint32_t IDESC_PV = umma::idesc_f16(FMT, 1, 0, 128, HQ);
+    constexpr uint32_t IDESC_PV = umma::idesc_f16(0u, 1, 0, 128, HQ);  // P V always in f16
     constexpr Smem L = smem_plan<FP8>();
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -471,7 +474,7 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
                         p0 *= tsc[j];
                         p1 *= tsc[j + 1];
                     }
-                    pw[j / 2] = pack2(p0, p1, FP8);
+                    pw[j / 2] = pack2(p0, p1, true);
                 }
                 lsum = lsum * alpha + rowsum;
                 uint8_t* prow = sm + L.p + sb * kPBytes;
@@ -480,15 +483,28 @@ __global__ void __launch_bounds__(FP8 ? 320 : 192, 1)
                     *reinterpret_cast<uint4*>(prow + sw64(h, c)) =
                         make_uint4(pw[4 * c], pw[4 * c + 1], pw[4 * c + 2], pw[4 * c + 3]);
             }
-            if (!fail && !FP8 && nvalid < kT) {
-                // rows past the last valid token hold stale page contents: zero their value
-                // columns so that P = 0 cannot meet a NaN/Inf
+            if (!fail && !FP8) {
+                // P V runs in f16 for both cache types: widen the tile's value columns (the
+                // first 512, boxes 0..7) from bf16 to f16 in place now that S has read them,
+                // saturating at +-65504; rows past the last valid token (stale page contents)
+                // become zeros so that P = 0 cannot meet a NaN/Inf
                 uint8_t* tile = sm + L.tiles + (size_t)ts * kTileBytes;
-                const int nr = kT - nvalid;
-                for (int i = tid; i < nr * 8 * 8; i += 128) {
-                    const int box = i / (nr * 8), rem = i - box * nr * 8;
-                    const int r = nvalid + rem / 8, c = rem & 7;
-                    *reinterpret_cast<uint4*>(tile + box * kBox + r * 128 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+                for (int i = tid; i < 8 * kT * 8; i += 128) {
+                    const int box = i / (kT * 8), rem = i - box * kT * 8;
+                    const int r = rem >> 3;
+                    uint4* ptr = reinterpret_cast<uint4*>(tile + box * kBox + r * 128 + (rem & 7) * 16);
+                    uint4 v = make_uint4(0u, 0u, 0u, 0u);
+                    if (r < nvalid) {
+                        const uint4 w = *ptr;
+                        const uint32_t ws[4] = {w.x, w.y, w.z, w.w};
+                        uint32_t o[4];
+#pragma unroll
+                        for (int e = 0; e < 4; e++)
+                            o[e] = pack2(fminf(fmaxf(bf16_lo(ws[e]), -65504.f), 65504.f),
+                                         fminf(fmaxf(bf16_hi(ws[e]), -65504.f), 65504.f), true);
+                        v = make_uint4(o[0], o[1], o[2], o[3]);
+                    }
+                    *ptr = v;
                 }
             }
             umma::fence_proxy_async_smem();
