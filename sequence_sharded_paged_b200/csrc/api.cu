@@ -146,7 +146,7 @@ cudaError_t launch_decode(const DecodeGeometry& g, const DecodeArgs& a, cudaStre
         case DecodePath::GqaMma:
             return launch_decode_gqa_mma(g, a, s);
         case DecodePath::MlaUmma:
-            return launch_decode_mla_umma(g, a, s);
+            return a.kv_scales ? launch_decode_mla_umma(g, a, s) : launch_decode_mla_bf16(g, a, s);
         default:
             return cudaErrorNotSupported;
     }

@@ -13,6 +13,45 @@ __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
+// Merge the split partials of the chunks of shard (u.n, u.b) for heads
+// h0..h0+nh-1 into o_partial / lse (executed by NT threads, tid in [0, NT)):
+//   M = max_j lse_j,  O = sum_j exp(lse_j - M) O_j / sum_j exp(lse_j - M),
+//   LSE = M + ln sum_j exp(lse_j - M).
+__device__ inline void merge_split_chunks(const DecodeArgs& a, const Unit& u, int64_t shard, int h0, int nh, int tid,
+                                          int NT) {
+    const int dv = a.dv;
+    const int K = u.n_chunks;
+    for (int i = tid; i < nh * (dv / 4); i += NT) {
+        const int h = i / (dv / 4), d4 = i - h * (dv / 4);
+        const float* lse_col = a.split_lse + (int64_t)u.slot_base * a.hq + h0 + h;
+        float M = -INFINITY;
+        for (int j = 0; j < K; j++) M = fmaxf(M, __ldcg(lse_col + (int64_t)j * a.hq));
+        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        float wsum = 0.f;
+        if (M != -INFINITY) {
+            for (int j = 0; j < K; j++) {
+                const float lj = __ldcg(lse_col + (int64_t)j * a.hq);
+                if (lj == -INFINITY) continue;
+                const float w = expf(lj - M);
+                wsum += w;
+                const float4 x = __ldcg(
+                    reinterpret_cast<const float4*>(a.split_o + ((int64_t)(u.slot_base + j) * a.hq + h0 + h) * dv) + d4);
+                o.x += w * x.x;
+                o.y += w * x.y;
+                o.z += w * x.z;
+                o.w += w * x.w;
+            }
+            const float inv = 1.f / wsum;
+            o.x *= inv;
+            o.y *= inv;
+            o.z *= inv;
+            o.w *= inv;
+        }
+        reinterpret_cast<float4*>(a.o_partial + (shard * a.hq + h0 + h) * dv)[d4] = o;
+        if (d4 == 0) a.lse[shard * a.hq + h0 + h] = (M == -INFINITY) ? -INFINITY : M + logf(wsum);
+    }
+}
+
 // Executed by the NT threads of barrier `bar_id` (tid in [0, NT)).
 //  sO   [nh][dv] normalised output of this unit for heads h0..h0+nh-1 (smem)
 //  sLse [nh]     natural-log LSE (-inf when the unit saw no token)
@@ -48,37 +87,7 @@ __device__ void finish_unit(const DecodeArgs& a, const Unit& u, int hb, int n_hb
     named_barrier_sync(bar_id, NT);
     if (!last) return;
     __threadfence();
-    const int K = u.n_chunks;
-    for (int i = tid; i < nh * (dv / 4); i += NT) {
-        int h = i / (dv / 4), d4 = i - h * (dv / 4);
-        const float* lse_col = a.split_lse + (int64_t)u.slot_base * a.hq + h0 + h;
-        float M = -INFINITY;
-        for (int j = 0; j < K; j++) M = fmaxf(M, __ldcg(lse_col + (int64_t)j * a.hq));
-        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
-        float wsum = 0.f;
-        if (M != -INFINITY) {
-            for (int j = 0; j < K; j++) {
-                float lj = __ldcg(lse_col + (int64_t)j * a.hq);
-                if (lj == -INFINITY) continue;
-                float w = expf(lj - M);
-                wsum += w;
-                float4 x = __ldcg(reinterpret_cast<const float4*>(
-                                      a.split_o + ((int64_t)(u.slot_base + j) * a.hq + h0 + h) * dv) +
-                                  d4);
-                o.x += w * x.x;
-                o.y += w * x.y;
-                o.z += w * x.z;
-                o.w += w * x.w;
-            }
-            float inv = 1.f / wsum;
-            o.x *= inv;
-            o.y *= inv;
-            o.z *= inv;
-            o.w *= inv;
-        }
-        reinterpret_cast<float4*>(a.o_partial + (shard * a.hq + h0 + h) * dv)[d4] = o;
-        if (d4 == 0) a.lse[shard * a.hq + h0 + h] = (M == -INFINITY) ? -INFINITY : M + logf(wsum);
-    }
+    merge_split_chunks(a, u, shard, h0, nh, tid, NT);
 }
 
 }  // namespace dcp

@@ -35,6 +35,9 @@ __device__ __forceinline__ void fence_proxy_async_smem() {
 // --- descriptors ------------------------------------------------------------
 enum Layout : uint64_t { kSw128 = 2, kSw64 = 4 };
 
+// 8-bit formats of kind::f8f6f4
+constexpr uint32_t kE4M3 = 0, kE5M2 = 1;
+
 // Shared-memory matrix descriptor: start address, leading / stride byte
 // offsets (bytes), swizzle layout; descriptor version 1 (sm_100).
 __device__ __forceinline__ uint64_t smem_desc(uint32_t saddr, uint32_t lbo, uint32_t sbo, Layout layout) {
@@ -50,6 +53,13 @@ __host__ __device__ constexpr uint32_t idesc_f16(uint32_t fmt, uint32_t a_major,
            ((M >> 4) << 24);
 }
 
+// Instruction descriptor of kind::f8f6f4 with fp32 accumulation (per-operand formats).
+__host__ __device__ constexpr uint32_t idesc_f8(uint32_t a_fmt, uint32_t b_fmt, uint32_t a_major, uint32_t b_major,
+                                                uint32_t M, uint32_t N) {
+    return (1u << 4) | (a_fmt << 7) | (b_fmt << 10) | (a_major << 15) | (b_major << 16) | ((N >> 3) << 17) |
+           ((M >> 4) << 24);
+}
+
 // --- MMA ---------------------------------------------------------------------
 __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
                                         uint32_t accumulate) {
@@ -57,6 +67,16 @@ __device__ __forceinline__ void mma_f16(uint32_t d_tmem, uint64_t a_desc, uint64
         "{\n\t.reg .pred p;\n\t"
         "setp.ne.b32 p, %4, 0;\n\t"
         "tcgen05.mma.cta_group::1.kind::f16 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
+        "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
+        : "memory");
+}
+
+__device__ __forceinline__ void mma_f8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                       uint32_t accumulate) {
+    asm volatile(
+        "{\n\t.reg .pred p;\n\t"
+        "setp.ne.b32 p, %4, 0;\n\t"
+        "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
         "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
         : "memory");
 }
