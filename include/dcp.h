@@ -187,6 +187,39 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
                               float* o_partial, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * DCP_STATIC_SCRATCH_BYTES -- size of the decode scratch built into the
+ * library: 64 MiB of device memory per device, reserved when the library's
+ * device code is loaded on that device.
+ */
+#define DCP_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+
+/*
+ * dcp_decode_partial_noalloc -- dcp_decode_partial with no caller workspace
+ * and no allocation: the plan, the split-chunk partials and the counters live
+ * in the library's built-in scratch (DCP_STATIC_SCRATCH_BYTES).
+ * The method's pages have no counterpart of this call.  It serves callers that
+ * cannot allocate device memory where they decode: a serving process whose
+ * caching allocator has already reserved the free HBM for its paged KV pool
+ * (a fresh cudaMalloc fails there, and the library has no handle on that
+ * allocator), and decode loops that cannot take the implicit device
+ * synchronisation of cudaMalloc / cudaFree.
+ *  Arguments as dcp_decode_partial, without ws / ws_bytes.
+ *  The plan is dcp_decode_partial's when dcp_decode_workspace_size() fits in
+ *  the scratch; otherwise the planner's split-slot bound is shrunk (fewer
+ *  units per CTA, so fewer, longer chunks) until it fits.  Returns
+ *  DCP_ERR_WORKSPACE_TOO_SMALL, launching nothing, when even the smallest
+ *  bound does not fit: the scratch grows with n_shards * B * hq (per-shard
+ *  counters) and with hq * dv (split partials).
+ *  The plan kernel, first on `stream`, clears the scratch's work ticket and
+ *  done counters; nothing else in it needs initialising.
+ *  Calls that can overlap in time (different streams, or threads without an
+ *  order between them) race on the one scratch array and give wrong results:
+ *  serialise them, e.g. on one stream.
+ */
+dcp_status dcp_decode_partial_noalloc(const dcp_cache_desc* cache, int32_t B, const void* q,
+                                      const int32_t* seq_lens, float* o_partial, float* lse, void* stream);
+
+/*
  * dcp_merge -- LSE-weighted merge of N partials (the arithmetic of the
  * all-gather + reduce-scatter step).
  * Passage: blog section 4.1 ("the LSE values reweight and merge the partials").

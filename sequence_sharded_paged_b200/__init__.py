@@ -9,7 +9,8 @@ fallback: if the library is missing, importing the entry points raises.
 
 Entry points (same names as ``include/dcp.h``): ``dcp_shard_counts``,
 ``dcp_shard_map``, ``dcp_kv_append``, ``dcp_decode_workspace_size``,
-``dcp_decode_partial``, ``dcp_merge``, ``dcp_get_device_status``.
+``dcp_decode_partial``, ``dcp_decode_partial_noalloc``, ``dcp_merge``,
+``dcp_get_device_status``.
 """
 from __future__ import annotations
 
@@ -34,7 +35,8 @@ DCP_BF16 = 0
 DCP_FP8_E4M3 = 1
 
 EXPORTED = ("dcp_status_string", "dcp_shard_counts", "dcp_shard_map", "dcp_kv_append",
-            "dcp_decode_workspace_size", "dcp_decode_partial", "dcp_merge", "dcp_get_device_status")
+            "dcp_decode_workspace_size", "dcp_decode_partial", "dcp_decode_partial_noalloc", "dcp_merge",
+            "dcp_get_device_status")
 
 
 class DcpError(RuntimeError):
@@ -77,10 +79,11 @@ def lib() -> ctypes.CDLL:
         L.dcp_decode_workspace_size.argtypes = [D, i32]
         L.dcp_decode_workspace_size.restype = ctypes.c_size_t
         L.dcp_decode_partial.argtypes = [D, i32, P, P, P, P, P, ctypes.c_size_t, P]
+        L.dcp_decode_partial_noalloc.argtypes = [D, i32, P, P, P, P, P]
         L.dcp_merge.argtypes = [i32, i32, i32, i32, P, P, P, P, P]
         L.dcp_get_device_status.argtypes = [ctypes.POINTER(i32), P]
-        for name in ("dcp_shard_counts", "dcp_shard_map", "dcp_kv_append", "dcp_decode_partial", "dcp_merge",
-                     "dcp_get_device_status"):
+        for name in ("dcp_shard_counts", "dcp_shard_map", "dcp_kv_append", "dcp_decode_partial",
+                     "dcp_decode_partial_noalloc", "dcp_merge", "dcp_get_device_status"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -141,6 +144,18 @@ def dcp_decode_partial(desc: CacheDesc, q, seq_lens, o_partial, lse, ws, stream=
     _check(lib().dcp_decode_partial(ctypes.byref(desc), q.shape[0], _ptr(q), _ptr(seq_lens), _ptr(o_partial),
                                     _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "dcp_decode_partial")
+
+
+# size of the library's built-in decode scratch (DCP_STATIC_SCRATCH_BYTES in dcp.h)
+DCP_STATIC_SCRATCH_BYTES = 64 << 20
+
+
+def dcp_decode_partial_noalloc(desc: CacheDesc, q, seq_lens, o_partial, lse, stream=None) -> None:
+    """dcp_decode_partial on the library's built-in scratch; allocates nothing.
+    Calls that can overlap in time race on that scratch."""
+    _check(lib().dcp_decode_partial_noalloc(ctypes.byref(desc), q.shape[0], _ptr(q), _ptr(seq_lens),
+                                            _ptr(o_partial), _ptr(lse), _stream(stream)),
+           "dcp_decode_partial_noalloc")
 
 
 def dcp_merge(o_partial, lse, out, lse_out=None, stream=None) -> None:

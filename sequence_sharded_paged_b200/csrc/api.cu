@@ -83,6 +83,83 @@ bool make_plan(const dcp_cache_desc* c, int B, int num_sms, Plan* p) {
     return true;
 }
 
+// ---------------------------------------------------------------------------
+// built-in decode scratch (dcp_decode_partial_noalloc)
+// ---------------------------------------------------------------------------
+// One per device context; its address is looked up once per device.
+static __device__ __align__(256) uint8_t g_decode_scratch[DCP_STATIC_SCRATCH_BYTES];
+
+uint8_t* g_scratch_ptr[kMaxDevices] = {nullptr};
+
+dcp_status decode_scratch(uint8_t** out) {
+    int dev = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DCP_ERR_CUDA;
+    std::lock_guard<std::mutex> lk(g_mu);
+    if (!g_scratch_ptr[dev]) {
+        void* p = nullptr;
+        if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess) return DCP_ERR_CUDA;
+        g_scratch_ptr[dev] = static_cast<uint8_t*>(p);
+    }
+    *out = g_scratch_ptr[dev];
+    return DCP_OK;
+}
+
+// make_plan's plan when its workspace fits in `cap` bytes; otherwise the same
+// geometry with half the units per CTA (a smaller chunk target, hence fewer
+// split slots), repeated down to one unit per CTA.  The bounds are make_plan's
+// for the smaller target.  False when nothing fits.
+bool make_plan_within(const dcp_cache_desc* c, int B, int num_sms, size_t cap, Plan* p) {
+    if (!make_plan(c, B, num_sms, p)) return false;
+    while (p->lay.total > cap && p->g.units_per_cta > 1) {
+        p->g.units_per_cta /= 2;
+        const int64_t target = (int64_t)p->g.units_per_cta * p->g.ctas;
+        const int64_t max_units = (int64_t)c->n_shards * B + target + 1;
+        p->lay = ws_layout(c->n_shards, B, c->hq, c->dv, (int)max_units, (int)(2 * target + 2));
+    }
+    return p->lay.total <= cap;
+}
+
+// The launch sequence of dcp_decode_partial (plan kernel, decode kernel) on a
+// workspace `w` laid out by `p`.
+dcp_status decode_on(const dcp_cache_desc* cache, int32_t B, const void* q, const int32_t* seq_lens,
+                     float* o_partial, float* lse, uint8_t* w, const Plan& p, int* status, cudaStream_t s) {
+    const int64_t target = (int64_t)p.g.units_per_cta * p.g.ctas;
+    cudaError_t e = launch_plan(seq_lens, B, cache->n_shards, cache->interleave, p.g.granule, p.g.min_chunk,
+                                (int)target, p.g.n_hb, w, p.lay.max_units, p.lay.max_split, cache->hq, cache->dv,
+                                status, s);
+    if (e != cudaSuccess) return DCP_ERR_CUDA;
+    DecodeArgs a;
+    a.k_pages = static_cast<const uint8_t*>(cache->k_pages);
+    a.v_pages = static_cast<const uint8_t*>(cache->v_pages);
+    a.kv_scales = cache->dtype == DCP_FP8_E4M3 ? cache->kv_scales : nullptr;
+    a.block_tables = cache->block_tables;
+    a.n_shards = cache->n_shards;
+    a.interleave = cache->interleave;
+    a.page_size = cache->page_size;
+    a.num_pages = cache->num_pages;
+    a.batch = B;
+    a.max_local_pages = cache->max_local_pages;
+    a.hq = cache->hq;
+    a.hkv = cache->hkv;
+    a.dk = cache->dk;
+    a.dv = cache->dv;
+    a.scale_log2 = cache->scale * kLog2e;
+    a.q = static_cast<const __nv_bfloat16*>(q);
+    a.seq_lens = seq_lens;
+    a.o_partial = o_partial;
+    a.lse = lse;
+    a.plan = reinterpret_cast<const PlanHeader*>(w);
+    a.ticket = &reinterpret_cast<PlanHeader*>(w)->next_unit;
+    a.units = reinterpret_cast<const Unit*>(w + p.lay.off_units);
+    a.done = reinterpret_cast<int32_t*>(w + p.lay.off_done);
+    a.split_o = reinterpret_cast<float*>(w + p.lay.off_split_o);
+    a.split_lse = reinterpret_cast<float*>(w + p.lay.off_split_lse);
+    a.status = status;
+    e = launch_decode(p.g, a, s);
+    if (e == cudaErrorNotSupported) return DCP_ERR_UNSUPPORTED;
+    return cuda_err(e);
+}
+
 }  // namespace
 
 // ---------------------------------------------------------------------------
@@ -291,6 +368,30 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
     e = launch_decode(p.g, a, s);
     if (e == cudaErrorNotSupported) return DCP_ERR_UNSUPPORTED;
     return cuda_err(e);
+}
+
+// No workspace argument and no allocation: for callers that cannot allocate
+// device memory where they decode (a serving process whose caching allocator
+// holds the free HBM for its KV pool; loops that cannot take cudaMalloc's
+// implicit synchronisation).  One scratch array per device: overlapping calls
+// race on it.
+dcp_status dcp_decode_partial_noalloc(const dcp_cache_desc* cache, int32_t B, const void* q,
+                                      const int32_t* seq_lens, float* o_partial, float* lse, void* stream) {
+    dcp_status st = check_desc(cache, true);
+    if (st != DCP_OK) return st;
+    if (B != cache->batch || !q || !seq_lens || !o_partial || !lse) return DCP_ERR_INVALID_ARG;
+    if (!aligned16(q) || !aligned16(o_partial) || !aligned16(lse)) return DCP_ERR_MISALIGNED;
+    int* status = nullptr;
+    int num_sms = 0;
+    st = device_info(&status, &num_sms);
+    if (st != DCP_OK) return st;
+    Plan p;
+    if (!make_plan(cache, B, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
+    if (!make_plan_within(cache, B, num_sms, DCP_STATIC_SCRATCH_BYTES, &p)) return DCP_ERR_WORKSPACE_TOO_SMALL;
+    uint8_t* w = nullptr;
+    st = decode_scratch(&w);
+    if (st != DCP_OK) return st;
+    return decode_on(cache, B, q, seq_lens, o_partial, lse, w, p, status, (cudaStream_t)stream);
 }
 
 dcp_status dcp_merge(int32_t N, int32_t B, int32_t H, int32_t Dv, const float* o_partial, const float* lse,
