@@ -223,7 +223,7 @@ cudaError_t launch_decode(const DecodeGeometry& g, const DecodeArgs& a, cudaStre
         case DecodePath::GqaMma:
             return launch_decode_gqa_mma(g, a, s);
         case DecodePath::MlaUmma:
-            return a.kv_scales ? launch_decode_mla_umma(g, a, s) : launch_decode_mla_bf16(g, a, s);
+            return a.kv_scales ? launch_decode_mla_fp8(g, a, s) : launch_decode_mla_bf16(g, a, s);
         default:
             return cudaErrorNotSupported;
     }

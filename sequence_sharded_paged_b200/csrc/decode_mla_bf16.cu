@@ -378,7 +378,9 @@ __global__ void __launch_bounds__(kThreads, 1)
                 s_alpha[h] = alpha;
             }
             if (threadIdx.x == 64) TRACE(7, seq);
-            // one barrier: some head rescaled while O^T holds data, or a wait failed
+            // one barrier: some head rescaled while O^T holds data, or a wait failed (a failing
+            // thread republishes the abort flag first, so every thread reads it set after the barrier)
+            if (fail) *s_abort = 1;
             const int any = named_barrier_or(kSmBar, 128, fail || (head && alpha != 1.f && o_has));
             if (threadIdx.x == 64) TRACE(8, seq);
             if (any && *s_abort) break;

@@ -61,6 +61,7 @@ bool mla_umma_supported(int hq, int page_size);
 size_t mla_umma_smem_bytes(bool fp8);
 cudaError_t launch_decode_mla_umma(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_mla_bf16(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s);
+cudaError_t launch_decode_mla_fp8(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s);
 
 cudaError_t launch_merge(int N, int B, int H, int Dv, const float* o_partial, const float* lse, float* out,
                          float* lse_out, cudaStream_t s);
