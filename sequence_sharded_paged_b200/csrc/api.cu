@@ -71,7 +71,18 @@ dcp_status check_desc(const dcp_cache_desc* c, bool need_pools) {
 struct Plan {
     DecodeGeometry g;
     WsLayout lay;
+    size_t off_qs = 0, off_qinv = 0;  // fp8 MLA query split (0 when unused)
 };
+
+// The fp8 MLA kernel reads the query split into two e4m3 terms from the end of
+// the workspace: [B][128 rows][576] bytes + [B][64] fp32 reciprocals.
+void add_query_split(const dcp_cache_desc* c, int B, Plan* p) {
+    p->off_qs = p->off_qinv = 0;
+    if (p->g.path != DecodePath::MlaUmma || c->dtype != DCP_FP8_E4M3) return;
+    p->off_qs = p->lay.total;
+    p->off_qinv = align256(p->off_qs + (size_t)B * 128 * 576);
+    p->lay.total = align256(p->off_qinv + (size_t)B * 64 * sizeof(float));
+}
 
 bool make_plan(const dcp_cache_desc* c, int B, int num_sms, Plan* p) {
     if (!decode_geometry(c->kind, c->dtype, c->hq, c->hkv, c->dk, c->dv, c->page_size, num_sms, &p->g)) return false;
@@ -80,6 +91,7 @@ bool make_plan(const dcp_cache_desc* c, int B, int num_sms, Plan* p) {
     const int64_t max_split = 2 * target + 2;
     if (max_units > (1 << 30)) return false;
     p->lay = ws_layout(c->n_shards, B, c->hq, c->dv, (int)max_units, (int)max_split);
+    add_query_split(c, B, p);
     return true;
 }
 
@@ -115,6 +127,7 @@ bool make_plan_within(const dcp_cache_desc* c, int B, int num_sms, size_t cap, P
         const int64_t target = (int64_t)p->g.units_per_cta * p->g.ctas;
         const int64_t max_units = (int64_t)c->n_shards * B + target + 1;
         p->lay = ws_layout(c->n_shards, B, c->hq, c->dv, (int)max_units, (int)(2 * target + 2));
+        add_query_split(c, B, p);
     }
     return p->lay.total <= cap;
 }
@@ -154,6 +167,8 @@ dcp_status decode_on(const dcp_cache_desc* cache, int32_t B, const void* q, cons
     a.done = reinterpret_cast<int32_t*>(w + p.lay.off_done);
     a.split_o = reinterpret_cast<float*>(w + p.lay.off_split_o);
     a.split_lse = reinterpret_cast<float*>(w + p.lay.off_split_lse);
+    a.qs = p.off_qs ? w + p.off_qs : nullptr;
+    a.qinv = p.off_qinv ? reinterpret_cast<float*>(w + p.off_qinv) : nullptr;
     a.status = status;
     e = launch_decode(p.g, a, s);
     if (e == cudaErrorNotSupported) return DCP_ERR_UNSUPPORTED;
@@ -364,6 +379,8 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
     a.done = reinterpret_cast<int32_t*>(w + p.lay.off_done);
     a.split_o = reinterpret_cast<float*>(w + p.lay.off_split_o);
     a.split_lse = reinterpret_cast<float*>(w + p.lay.off_split_lse);
+    a.qs = p.off_qs ? w + p.off_qs : nullptr;
+    a.qinv = p.off_qinv ? reinterpret_cast<float*>(w + p.off_qinv) : nullptr;
     a.status = status;
     e = launch_decode(p.g, a, s);
     if (e == cudaErrorNotSupported) return DCP_ERR_UNSUPPORTED;

@@ -249,6 +249,8 @@ struct DecodeArgs {
     int32_t* done;
     float* split_o;
     float* split_lse;
+    uint8_t* qs;         // fp8 MLA: query rows split into two e4m3 terms [B][128][576] (else null)
+    float* qinv;         // fp8 MLA: 1 / sigma per (request, head) [B][64] (else null)
     int* status;
 };
 

@@ -9,32 +9,42 @@
 //
 // Value of a latent element = e4m3 code * s_t (s_t = per-token scale).
 //
-// Scores.  Each head's bf16 query row is scaled by a power of two sigma_h
-// (largest |q| sigma_h in [128, 256)) and split exactly into two e4m3 terms,
-// q sigma_h = q_hi + q_lo (bf16 has 8 significant bits, e4m3 4; only elements
-// below ~2^-17 of the row maximum lose bits).  The two terms are stacked as
-// the 128 rows of one operand:
-//   [S_hi; S_lo] = [Q_hi; Q_lo] . C^T   M = 128, N = 64 tokens, K = 576 (e4m3 x e4m3)
-// so 18 MMAs per 64-token tile read the raw page.  Lanes 0..63 of TMEM hold
-// S_hi, lanes 64..127 S_lo; the softmax warps exchange halves through shared
-// memory and form s = scale * s_t * (S_hi + S_lo) / sigma_h.
+// Query.  A small kernel splits each head's bf16 query row exactly into two
+// e4m3 terms after scaling it by a power of two sigma_h (largest |q| sigma_h in
+// [128, 256)): q sigma_h = q_hi + q_lo (bf16 has 8 significant bits, e4m3 4;
+// only elements below ~2^-17 of the row maximum lose bits).  Rows are stacked
+// 128 high: for heads 16 j .. 16 j + 15, rows 32 j .. 32 j + 15 hold q_hi and
+// rows 32 j + 16 .. 32 j + 31 hold q_lo, so that a head's two score rows land
+// in one warp's TMEM lane quadrant.  The first 512 columns of those rows live
+// in tensor memory (the MMA's A operand), the 64 rope columns in shared memory.
 //
-// Values.  O^T = V^T . P'^T with V^T read MN-major straight from the raw tile
-// (e4m3) and P' = 16 * p * s_t split into three e5m2 terms (about nine
-// significant bits: relative error below 2^-9 of P, inside the fp8 tolerance;
-// e5m2's exponent range covers p * s_t without per-token rescaling):
-//   O^T += V^T . P'_j^T   M = 128 value columns (4 blocks), N = Hq, K = 64, j = 0..2
-// 24 MMAs per tile.  O = O^T / (16 * l).  The running maximum is rescaled
-// lazily (O^T only when a head's maximum grows by more than 2^8).
+// Scores.  [S_hi; S_lo] = [Q_hi; Q_lo] . C^T, M = 128, N = 128 tokens, K = 576:
+// 16 MMAs with A in TMEM + 2 with A in shared memory; the two pages of the tile
+// are the only shared-memory operand.  Lane pairs (l, l + 16) swap halves with
+// shuffles and form s = scale * s_t * (S_hi + S_lo) / sigma_h.
 //
-// Tiles: one 64-token page per tile, nine [64 rows][64 B] TMA boxes with
-// 64-byte swizzle (36 KB) + 256 B of scales; three stages in flight.
+// Values.  O^T = V^T . W^T with V^T read MN-major straight from the raw pages
+// and W = p * s_t in two e4m3 terms (relative error below 2^-8).  The running
+// maximum m absorbs the tile's largest scale (m >= max_t (x_t + log2 s_t), x in
+// log2 units), so W = 2^(x - m) s_t <= 2^8 stays inside e4m3's range whatever
+// the scales; it is rescaled lazily (O^T only when m grows by more than 2^8).
+//   O^T += V^T . W_j^T   M = 128 value columns (4 blocks), N = Hq, K = 128, j = 0, 1
+// 32 MMAs per tile.  O = O^T / l with l = sum_t 2^(x_t - m).
+//
+// Tiles: two 64-token pages (128 tokens).  Each page arrives as nine
+// [64 rows][64 B] TMA boxes with 64-byte swizzle (36 KB) + 256 B of scales;
+// block kb of the four page slots is contiguous, so that the two pages of a
+// tile form one 128-row operand.  Two tiles in flight.
 //
 // Warp roles (one CTA per SM, persistent, units from an atomic ticket):
 //   warp 0      TMA producer (lane 0)
 //   warp 1      TMEM allocation, MMA issue (lane 0, event loop)
-//   warps 2..5  q split, softmax, lazy rescale of O^T, epilogue; the warp on TMEM
-//               quadrant q owns heads 32 (q & 1) .. +31 and tokens 32 (q >> 1) .. +31
+//   warps 2..9  query rows, softmax, lazy rescale of O^T, epilogue.  The two
+//               warps on TMEM quadrant j own heads 16 j .. 16 j + 15: warp
+//               group g (warps 2..5: g = 0, 6..9: g = 1) the tile's tokens
+//               64 g .. 64 g + 63, in which lane l < 16 takes the first 32
+//               and lane l + 16 the last 32; g also picks the value blocks
+//               2 g, 2 g + 1 that the warp rescales and stores.
 #include "common.cuh"
 #include "finish.cuh"
 #include "kernels.h"
@@ -43,45 +53,72 @@
 
 namespace dcp {
 
+// Optional timeline of CTA 0 (SM clock at each protocol step), compiled only
+// with -DDCP_TRACE for profiling builds; expands to nothing otherwise.
+#ifdef DCP_TRACE
+__device__ unsigned long long g_mla8_trace[16][512];
+#define TRACE(ev, k)                                                          \
+    do {                                                                      \
+        if (blockIdx.x == 0 && (k) < 512) g_mla8_trace[ev][(k)] = clock64();  \
+    } while (0)
+extern "C" int dcp_trace8_read(unsigned long long* host) {
+    return (int)cudaMemcpyFromSymbol(host, g_mla8_trace, sizeof(g_mla8_trace));
+}
+#else
+#define TRACE(ev, k) \
+    do {             \
+    } while (0)
+#endif
+
 namespace {
 
-constexpr int kT = 64;                     // tokens per tile (one page)
+constexpr int kPg = 64;                    // tokens per page
+constexpr int kT = 128;                    // tokens per tile (two pages)
 constexpr int kKB = 9;                     // 576 = 9 blocks of 64 bytes
-constexpr int kBox = kT * 64;              // [64 rows][64 B] box: 4 KB
-constexpr int kTileBytes = kKB * kBox;     // 36864
-constexpr int kQBox = 128 * 64;            // [128 rows][64 B]: 8 KB
-constexpr int kQBytes = kKB * kQBox;       // 73728
-constexpr int kStages = 3;
-constexpr int kPTerm = 64 * 64;            // P'_j^T [64 heads][64 tokens] e5m2: 4 KB
-constexpr int kPBuf = 3 * kPTerm;          // 12 KB
+constexpr int kBox = kPg * 64;             // [64 rows][64 B] box of one page: 4 KB
+constexpr int kSlots = 5;                  // page slots: two and a half tiles in flight
+constexpr int kKbStride = kSlots * kBox;   // block kb of every slot: [slot][64 rows][64 B]
+constexpr int kPageBytes = kKB * kBox;     // 36864
+constexpr int kRopeBytes = 128 * 64;       // rope columns of the 128 query rows
+constexpr int kPTerm = 64 * 128;           // W_j^T [2 pages][64 heads][64 tokens] e4m3: 8 KB
+constexpr int kPBuf = 2 * kPTerm;          // 16 KB
 constexpr float kRescaleLog2 = 8.f;
-constexpr float kPScale = 16.f;            // P' = 16 p s_t
-constexpr int kSmBar = 1;
-constexpr int kThreads = 192;
+constexpr int kSmBar = 1;                  // the 256 softmax threads
+constexpr int kPairBar = 2;                // + quadrant: the two warps sharing a TMEM lane quadrant
+constexpr int kSoftWarps = 8;
+constexpr int kThreads = 32 * (2 + kSoftWarps);
+constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384;  // TMEM columns
 
-constexpr uint32_t kOffQ = 0;
-constexpr uint32_t kOffTiles = kQBytes;
-constexpr uint32_t kOffScales = kOffTiles + kStages * kTileBytes;
-constexpr uint32_t kOffP = (kOffScales + kStages * kT * 4 + 1023) / 1024 * 1024;
-constexpr uint32_t kOffX = kOffP + 2 * kPBuf;                 // [2 halves][64 heads][32] f32
-constexpr uint32_t kOffXmax = kOffX + 2 * 64 * 32 * 4;        // [2][64] f32
-constexpr uint32_t kOffBars = kOffXmax + 2 * 64 * 4;
+constexpr uint32_t kOffTiles = 0;
+constexpr uint32_t kOffRope = kOffTiles + kKB * kKbStride;
+constexpr uint32_t kOffP = kOffRope + kRopeBytes;
+constexpr uint32_t kOffScales = kOffP + 2 * kPBuf;
+constexpr uint32_t kOffBars = kOffScales + kSlots * kPg * 4;
 constexpr uint32_t kOffMeta = kOffBars + 32 * 8;
-constexpr uint32_t kOffSmall = kOffMeta + kStages * 16;
-constexpr uint32_t kSmemBytes = kOffSmall + (6 * 64 + 16) * 4 + 1024;
+constexpr uint32_t kOffSmall = kOffMeta + kSlots * 16;
+// s_alpha[64], s_inv[64], s_gmax[2][64], s_gsmax[2][64], s_gl[2][64], misc[16]
+constexpr uint32_t kSmemBytes = kOffSmall + (8 * 64 + 16) * 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
+static_assert(kOffRope % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands need 1 KB alignment");
 
 enum : int {
-    B_TILE_FULL = 0,   // [3]
-    B_TILE_EMPTY = 3,  // [3]
-    B_S_FULL = 6,      // [2]
-    B_P_FULL = 8,      // [2]
-    B_PV_DONE = 10,    // [2]
-    B_Q_FULL = 12,
-    B_Q_FREE = 13,
-    B_O_FREE = 14,
-    B_FINAL = 15,
+    B_PAGE_FULL = 0,    // [kSlots]
+    B_PAGE_EMPTY = 8,   // [kSlots]
+    B_S_FULL = 16,
+    B_S_FREE = 17,
+    B_P_FULL = 18,      // [2]
+    B_PV_DONE = 20,     // [2]
+    B_Q_FULL = 22,
+    B_Q_FREE = 23,
+    B_O_FREE = 24,
+    B_FINAL = 25,
 };
+
+// Tile k occupies page slots (2k) mod 5 and (2k + 1) mod 5; page p of the ring
+// sequence completes phase (p / 5) & 1 of its slot's barriers.
+__device__ __forceinline__ int slot_of(uint32_t page_seq) { return (int)(page_seq % kSlots); }
+__device__ __forceinline__ uint32_t phase_of(uint32_t page_seq) { return (page_seq / kSlots) & 1; }
+
 
 // byte offset of 16-byte chunk c (0..3) of row r in a 64-byte-swizzled block
 __device__ __forceinline__ uint32_t sw64(int r, int c) { return (uint32_t)(r * 64 + (((c ^ (r >> 1)) & 3) << 4)); }
@@ -99,148 +136,248 @@ __device__ __forceinline__ int named_barrier_or(int id, int nthreads, int pred) 
     return r;
 }
 
-// two floats -> two 8-bit codes (round to nearest even, saturating to the largest finite value)
-__device__ __forceinline__ uint32_t to_e4m3x2(float a, float b) {
+// two floats -> two e4m3 codes (round to nearest even, saturating)
+__device__ __forceinline__ uint32_t f32x2_to_e4m3x2(float a, float b) {
     return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E4M3);
 }
-__device__ __forceinline__ uint32_t to_e5m2x2(float a, float b) {
-    return (uint32_t)__nv_cvt_float2_to_fp8x2(make_float2(a, b), __NV_SATFINITE, __NV_E5M2);
-}
-__device__ __forceinline__ float2 from_fp8x2(uint32_t c, __nv_fp8_interpretation_t k) {
-    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(c & 0xFFFF), k);
+__device__ __forceinline__ float2 e4m3x2_to_f32x2(uint32_t c) {
+    __half2_raw h = __nv_cvt_fp8x2_to_halfraw2((__nv_fp8x2_storage_t)(c & 0xFFFF), __NV_E4M3);
     return __half22float2(*reinterpret_cast<__half2*>(&h));
 }
+// w0, w1 >= 0 -> two-term e4m3 codes (hi, lo) with w ~ hi + lo, via f16 (11 bits)
+__device__ __forceinline__ void split_e4m3x2(float w0, float w1, uint32_t& hi, uint32_t& lo) {
+    const __half2 h = __floats2half2_rn(w0, w1);
+    const __nv_fp8x2_storage_t c =
+        __nv_cvt_halfraw2_to_fp8x2(*reinterpret_cast<const __half2_raw*>(&h), __NV_SATFINITE, __NV_E4M3);
+    __half2_raw br = __nv_cvt_fp8x2_to_halfraw2(c, __NV_E4M3);
+    const __half2 r = __hsub2(h, *reinterpret_cast<__half2*>(&br));  // exact
+    hi = (uint32_t)c;
+    lo = (uint32_t)__nv_cvt_halfraw2_to_fp8x2(*reinterpret_cast<const __half2_raw*>(&r), __NV_SATFINITE, __NV_E4M3);
+}
+// 32 weights -> two e4m3 terms, four codes per word
+__device__ __forceinline__ void split32(const float (&w)[32], uint32_t (&chi)[8], uint32_t (&clo)[8]) {
+#pragma unroll
+    for (int j = 0; j < 32; j += 4) {
+        uint32_t h01, l01, h23, l23;
+        split_e4m3x2(w[j], w[j + 1], h01, l01);
+        split_e4m3x2(w[j + 2], w[j + 3], h23, l23);
+        chi[j / 4] = h01 | (h23 << 16);
+        clo[j / 4] = l01 | (l23 << 16);
+    }
+}
 
+// ------------------------------------------------------------------------------------------
+// Query split: one warp per (request, head).  Writes rows hi / lo of qs[b][128][576] and
+// qinv[b][64] = 1 / sigma_h.
+__global__ void __launch_bounds__(128) mla_fp8_qsplit_kernel(const __nv_bfloat16* __restrict__ q, int B, int HQ,
+                                                             uint8_t* __restrict__ qs, float* __restrict__ qinv) {
+    const int gw = (int)((blockIdx.x * blockDim.x + threadIdx.x) >> 5), lane = threadIdx.x & 31;
+    if (gw >= B * HQ) return;
+    const int b = gw / HQ, h = gw - b * HQ;
+    const uint4* qrow = reinterpret_cast<const uint4*>(q + ((int64_t)b * HQ + h) * 576);
+    // lane handles 16-element chunks c = lane and c = lane + 32 (< 36)
+    uint4 w[2][2];
+    float amax = 0.f;
+#pragma unroll
+    for (int k2 = 0; k2 < 2; k2++) {
+        const int c = lane + 32 * k2;
+        if (c < 36) {
+            w[k2][0] = __ldg(qrow + 2 * c);
+            w[k2][1] = __ldg(qrow + 2 * c + 1);
+            const uint32_t ws[8] = {w[k2][0].x, w[k2][0].y, w[k2][0].z, w[k2][0].w,
+                                    w[k2][1].x, w[k2][1].y, w[k2][1].z, w[k2][1].w};
+#pragma unroll
+            for (int e = 0; e < 8; e++) amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(ws[e])), fabsf(bf16_hi(ws[e]))));
+        }
+    }
+#pragma unroll
+    for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
+    int ex = 0;
+    frexpf(amax, &ex);      // amax in [2^(ex-1), 2^ex)
+    ex = max(ex, -110);     // sigma and 1/sigma stay finite
+    const float sig = amax > 0.f ? ldexpf(1.f, 8 - ex) : 1.f;
+    if (lane == 0) qinv[(int64_t)b * 64 + h] = 1.f / sig;
+    uint8_t* hi_row = qs + ((int64_t)b * 128 + 32 * (h >> 4) + (h & 15)) * 576;
+    uint8_t* lo_row = hi_row + 16 * 576;
+#pragma unroll
+    for (int k2 = 0; k2 < 2; k2++) {
+        const int c = lane + 32 * k2;
+        if (c < 36) {
+            const uint32_t ws[8] = {w[k2][0].x, w[k2][0].y, w[k2][0].z, w[k2][0].w,
+                                    w[k2][1].x, w[k2][1].y, w[k2][1].z, w[k2][1].w};
+            uint32_t hi[4], lo[4];
+#pragma unroll
+            for (int e = 0; e < 4; e++) {
+                const float a0 = bf16_lo(ws[2 * e]) * sig, a1 = bf16_hi(ws[2 * e]) * sig;
+                const float a2 = bf16_lo(ws[2 * e + 1]) * sig, a3 = bf16_hi(ws[2 * e + 1]) * sig;
+                const uint32_t h01 = f32x2_to_e4m3x2(a0, a1), h23 = f32x2_to_e4m3x2(a2, a3);
+                const float2 d01 = e4m3x2_to_f32x2(h01), d23 = e4m3x2_to_f32x2(h23);
+                hi[e] = h01 | (h23 << 16);
+                lo[e] = f32x2_to_e4m3x2(a0 - d01.x, a1 - d01.y) | (f32x2_to_e4m3x2(a2 - d23.x, a3 - d23.y) << 16);
+            }
+            *reinterpret_cast<uint4*>(hi_row + 16 * c) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
+            *reinterpret_cast<uint4*>(lo_row + 16 * c) = make_uint4(lo[0], lo[1], lo[2], lo[3]);
+        }
+    }
+}
+
+// ------------------------------------------------------------------------------------------
 template <int HQ>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_fp8_kernel(const __grid_constant__ CUtensorMap tmC, DecodeArgs a) {
-    constexpr uint32_t IDESC_S = umma::idesc_f8(umma::kE4M3, umma::kE4M3, 0, 0, 128, kT);
-    constexpr uint32_t IDESC_PV = umma::idesc_f8(umma::kE4M3, umma::kE5M2, 1, 0, 128, HQ);
+    constexpr uint32_t IDESC_S128 = umma::idesc_f8(umma::kE4M3, umma::kE4M3, 0, 0, 128, 128);
+    constexpr uint32_t IDESC_S64 = umma::idesc_f8(umma::kE4M3, umma::kE4M3, 0, 0, 128, 64);
+    constexpr uint32_t IDESC_PV = umma::idesc_f8(umma::kE4M3, umma::kE4M3, 1, 0, 128, HQ);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kOffBars);
-    StageMeta* tmeta = reinterpret_cast<StageMeta*>(sm + kOffMeta);
-    float* xbuf = reinterpret_cast<float*>(sm + kOffX);
-    float* xmax = reinterpret_cast<float*>(sm + kOffXmax);
-    float* s_m = reinterpret_cast<float*>(sm + kOffSmall);
-    float* s_l0 = s_m + 64;
-    float* s_l1 = s_l0 + 64;
-    float* s_alpha = s_l1 + 64;
-    float* s_qs = s_alpha + 64;   // 1 / sigma_h
-    int* s_misc = reinterpret_cast<int*>(s_qs + 128);  // [0] tmem base, [2] split flag, [3] abort
+    StageMeta* tmeta = reinterpret_cast<StageMeta*>(sm + kOffMeta);  // per page slot (a tile's first)
+    float* s_alpha = reinterpret_cast<float*>(sm + kOffSmall);
+    float* s_inv = s_alpha + 64;
+    float* s_gmax = s_inv + 64;     // [2 token groups][64 heads]
+    float* s_gsmax = s_gmax + 128;  // [2][64]
+    float* s_gl = s_gsmax + 128;    // [2][64]
+    int* s_misc = reinterpret_cast<int*>(s_gl + 128);  // [0] tmem base, [2] split flag, [3] abort
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_misc + 3);
 
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t sm_u32 = smem_u32(sm);
 
     if (threadIdx.x == 0) {
-        for (int i = 0; i < kStages; i++) {
-            mbar_init(bar + B_TILE_FULL + i, 1);
-            mbar_init(bar + B_TILE_EMPTY + i, 1);
+        for (int i = 0; i < kSlots; i++) {
+            mbar_init(bar + B_PAGE_FULL + i, 1);
+            mbar_init(bar + B_PAGE_EMPTY + i, 1);
         }
         for (int i = 0; i < 2; i++) {
-            mbar_init(bar + B_S_FULL + i, 1);
-            mbar_init(bar + B_P_FULL + i, 4);
+            mbar_init(bar + B_P_FULL + i, kSoftWarps);
             mbar_init(bar + B_PV_DONE + i, 1);
         }
-        mbar_init(bar + B_Q_FULL, 4);
+        mbar_init(bar + B_S_FULL, 1);
+        mbar_init(bar + B_S_FREE, kSoftWarps);
+        mbar_init(bar + B_Q_FULL, kSoftWarps);
         mbar_init(bar + B_Q_FREE, 1);
-        mbar_init(bar + B_O_FREE, 4);
+        mbar_init(bar + B_O_FREE, kSoftWarps);
         mbar_init(bar + B_FINAL, 1);
         *s_abort = 0;
         fence_barrier_init();
     }
-    // Q rows of heads >= HQ stay zero for the whole kernel
-    for (int i = threadIdx.x; i < kQBytes / 16; i += blockDim.x)
-        reinterpret_cast<uint4*>(sm + kOffQ)[i] = make_uint4(0u, 0u, 0u, 0u);
+    // rope rows of heads >= HQ stay zero for the whole kernel
+    for (int i = threadIdx.x; i < kRopeBytes / 16; i += blockDim.x)
+        reinterpret_cast<uint4*>(sm + kOffRope)[i] = make_uint4(0u, 0u, 0u, 0u);
     if (warp == 1) umma::tmem_alloc(reinterpret_cast<uint32_t*>(s_misc), 512);
     umma::fence_proxy_async_smem();
     umma::fence_before_sync();
     __syncthreads();
     umma::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(s_misc);
-    const uint32_t t_o = tmem;         // O^T: columns [blk*HQ, blk*HQ + HQ)
-    const uint32_t t_s = tmem + 256;   // S buffers: [256 + 64 sb, +64)
+    const uint32_t t_o = tmem + kColO;  // O^T: columns [blk*HQ, blk*HQ + HQ)
+    const uint32_t t_s = tmem + kColS;  // S: 128 token columns
+    const uint32_t t_q = tmem + kColQ;  // query rows, first 512 columns (128 TMEM columns)
     const int num_units = a.plan->num_units;
     const int P = a.page_size;
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
-        if (lane == 0) {
-            const uint64_t pol = l2_policy_evict_first();
-            tma_prefetch_desc(&tmC);
-            int stage = 0, issued = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            while (ok) {
-                const int ui = atomicAdd(a.ticket, 1);
-                const bool done = ui >= num_units;
-                Unit u;
-                int nt = 1;
-                if (!done) {
-                    u = a.units[ui];
-                    nt = (u.t1 - u.t0 + kT - 1) / kT;
+        // Pages go into the slot ring one by one, each as soon as its slot is free.  One
+        // tile of lookahead: the next tile's unit and page indices are fetched before the
+        // waits, so their latency overlaps them.  Lane 0 takes tickets and handles the
+        // barriers; lanes 0..8 then issue a page's nine boxes and lane 9 its scales at once.
+        const uint64_t pol = l2_policy_evict_first();
+        if (lane == 0) tma_prefetch_desc(&tmC);
+        int ui = -1, k = 0, nt = 0;
+        Unit u;
+        u.n = u.b = u.t0 = u.t1 = u.slot = u.n_chunks = u.slot_base = u.pad = 0;
+        // moves (ui, k) to the next tile (the same on every lane); false when no work is left
+        auto advance = [&]() -> bool {
+            if (ui >= 0 && k + 1 < nt) {
+                k++;
+                return true;
+            }
+            int nu = 0;
+            if (lane == 0) nu = atomicAdd(a.ticket, 1);
+            ui = __shfl_sync(0xffffffffu, nu, 0);
+            if (ui >= num_units) return false;
+            u = a.units[ui];
+            nt = max(1, (u.t1 - u.t0 + kT - 1) / kT);  // an empty unit still yields one tile
+            k = 0;
+            return true;
+        };
+        auto pages = [&](int& p0, int& p1) {
+            const int t = u.t0 + k * kT;
+            const int nv = max(0, min(u.t1 - t, kT));
+            p0 = nv > 0 ? page_of(a, u.n, u.b, t / P) : -1;
+            p1 = nv > kPg ? page_of(a, u.n, u.b, t / P + 1) : -1;
+        };
+        bool have = advance();
+        int pg0 = -1, pg1 = -1;
+        if (have) pages(pg0, pg1);
+        uint32_t ps = 0;  // pages issued into the ring
+        bool ok = true;
+        while (ok) {
+            const bool c_have = have;
+            const int c_ui = ui, c_k = k, c_nt = nt, c_pg0 = pg0, c_pg1 = pg1;
+            const Unit c_u = u;
+            if (have) {
+                have = advance();
+                if (have) pages(pg0, pg1);
+            }
+            const int t = c_u.t0 + c_k * kT;
+            int nvalid = c_have ? max(0, min(c_u.t1 - t, kT)) : 0;
+            const int npages = (nvalid + kPg - 1) / kPg;
+            if ((npages > 0 && c_pg0 < 0) || (npages > 1 && c_pg1 < 0)) {
+                if (lane == 0) record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
+                nvalid = 0;
+            }
+            const int flags = (c_k == 0 ? kStageFirst : 0) | (c_k == c_nt - 1 ? kStageLast : 0);
+            for (int g = 0; g < 2; g++, ps++) {
+                const int slot = slot_of(ps);
+                int waited = 1;
+                if (lane == 0) waited = mbar_wait(bar + B_PAGE_EMPTY + slot, phase_of(ps) ^ 1, s_abort, a.status);
+                if (!__shfl_sync(0xffffffffu, waited, 0)) {
+                    ok = false;
+                    break;
                 }
-                int k = 0;
-                do {
-                    if (!mbar_wait(bar + B_TILE_EMPTY + stage, phase ^ 1, s_abort, a.status)) {
+                if (lane == 0) TRACE(14, ps / 2);
+                if (g == 0) {
+                    if (lane == 0)
+                        tmeta[slot] = c_have ? StageMeta{c_ui, t, flags | (nvalid << 8), c_k} : StageMeta{-1, 0, 0, 0};
+                    if (!c_have) {
+                        if (lane == 0) mbar_arrive(bar + B_PAGE_FULL + slot);
                         ok = false;
                         break;
                     }
-                    if (done) {
-                        tmeta[stage] = StageMeta{-1, 0, 0, 0};
-                        mbar_arrive(bar + B_TILE_FULL + stage);
-                        ok = false;
-                        break;
-                    }
-                    const int t = u.t0 + k * kT;
-                    const int nvalid = nt == 0 ? 0 : min(u.t1 - t, kT);
-                    const int flags = (k == 0 ? kStageFirst : 0) | (k >= nt - 1 ? kStageLast : 0);
-                    int pg = -1;
-                    if (nt > 0) {
-                        pg = page_of(a, u.n, u.b, t / P);
-                        if (pg < 0) record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
-                    }
-                    tmeta[stage] = StageMeta{ui, t, flags | ((pg >= 0 ? nvalid : 0) << 8), k};
-                    if (pg >= 0) {
-                        mbar_arrive_expect_tx(bar + B_TILE_FULL + stage, kTileBytes + kT * 4);
-                        uint8_t* dst = sm + kOffTiles + (size_t)stage * kTileBytes;
-                        const int32_t row0 = pg * P + (t % P);
-#pragma unroll
-                        for (int kb = 0; kb < kKB; kb++)
-                            tma_load_2d(dst + kb * kBox, &tmC, kb * 64, row0, bar + B_TILE_FULL + stage, pol);
-                        bulk_g2s(sm + kOffScales + stage * kT * 4, a.kv_scales + row0, kT * 4,
-                                 bar + B_TILE_FULL + stage);
-                    } else {
-                        mbar_arrive(bar + B_TILE_FULL + stage);
-                    }
-                    issued++;
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
-                    k++;
-                } while (k < nt);
-            }
-            if (*s_abort) {  // bounded drain of copies still in flight
-                int n = issued < kStages ? issued : kStages;
-                for (int i = 0; i < n; i++) {
-                    stage = stage == 0 ? kStages - 1 : stage - 1;
-                    if (stage == kStages - 1) phase ^= 1;
-                    mbar_wait(bar + B_TILE_FULL + stage, phase, nullptr, a.status);
                 }
+                if (nvalid > g * kPg) {
+                    if (lane == 0) mbar_arrive_expect_tx(bar + B_PAGE_FULL + slot, kPageBytes + kPg * 4);
+                    __syncwarp();
+                    const int32_t row0 = (g ? c_pg1 : c_pg0) * P;
+                    if (lane < kKB)
+                        tma_load_2d(sm + kOffTiles + slot * kBox + lane * kKbStride, &tmC, lane * 64, row0,
+                                    bar + B_PAGE_FULL + slot, pol);
+                    else if (lane == kKB)
+                        bulk_g2s(sm + kOffScales + slot * kPg * 4, a.kv_scales + row0, kPg * 4,
+                                 bar + B_PAGE_FULL + slot);
+                } else if (lane == 0) {
+                    mbar_arrive(bar + B_PAGE_FULL + slot);
+                }
+                if (lane == 0) TRACE(15, ps / 2);
             }
+        }
+        if (lane == 0 && *s_abort) {  // bounded drain of copies still in flight
+            const uint32_t n = ps < (uint32_t)kSlots ? ps : (uint32_t)kSlots;
+            for (uint32_t i = 1; i <= n; i++)
+                mbar_wait(bar + B_PAGE_FULL + slot_of(ps - i), phase_of(ps - i), nullptr, a.status);
         }
     } else if (warp == 1) {
         // ------------------------------------------------------------------ MMA issuer (event loop)
         if (lane == 0) {
-            const uint64_t dq0 = umma::smem_desc(sm_u32 + kOffQ, 16, 512, umma::kSw64);
+            const uint64_t dr0 = umma::smem_desc(sm_u32 + kOffRope, 16, 512, umma::kSw64);
             const uint64_t dt0 = umma::smem_desc(sm_u32 + kOffTiles, 16, 512, umma::kSw64);
-            const uint64_t dv0 = umma::smem_desc(sm_u32 + kOffTiles, kBox, 512, umma::kSw64);
+            const uint64_t dv0 = umma::smem_desc(sm_u32 + kOffTiles, kKbStride, 512, umma::kSw64);
             const uint64_t dp0 = umma::smem_desc(sm_u32 + kOffP, 16, 512, umma::kSw64);
             uint32_t next_s = 0, next_pv = 0, unit_k = 0, ofree_k = 0;
-            uint32_t first_bits = 0;  // bit b: the tile in S buffer b opened its unit
+            uint32_t first_bits = 0;  // bit b: tile with parity b opened its unit
             bool sentinel = false;
             uint64_t t_prog = global_timer_ns();
             while (true) {
@@ -251,50 +388,89 @@ __global__ void __launch_bounds__(kThreads, 1)
                     if (mbar_test(bar + B_P_FULL + pb, (next_pv >> 1) & 1) &&
                         (!fst || mbar_test(bar + B_O_FREE, (ofree_k & 1) ^ 1))) {
                         if (fst) ofree_k++;
+                        TRACE(2, next_pv);
                         umma::fence_after_sync();
-                        const int st = next_pv % kStages;
-                        const uint64_t tile = (uint64_t)((st * kTileBytes) >> 4);
-                        const uint64_t pbuf = (uint64_t)((pb * kPBuf) >> 4);
+                        // page by page, so that the first page's slot is released early; consecutive
+                        // MMAs go to different accumulator blocks
 #pragma unroll
-                        for (int j = 0; j < 3; j++)
+                        for (int g = 0; g < 2; g++) {
+                            const int sl = slot_of(2 * next_pv + g);
 #pragma unroll
-                            for (int blk = 0; blk < 4; blk++)
+                            for (int j = 0; j < 2; j++)
 #pragma unroll
-                                for (int ks = 0; ks < 2; ks++) {
-                                    const uint64_t ad = dv0 + tile + (uint64_t)(((2 * blk) * kBox + ks * 2048) >> 4);
-                                    const uint64_t bd = dp0 + pbuf + (uint64_t)((j * kPTerm + ks * 32) >> 4);
-                                    umma::mma_f8(t_o + blk * HQ, ad, bd, IDESC_PV, (fst && j == 0 && ks == 0) ? 0u : 1u);
-                                }
+                                for (int ks = 0; ks < 2; ks++)
+#pragma unroll
+                                    for (int blk = 0; blk < 4; blk++) {
+                                        const uint64_t ad =
+                                            dv0 + (uint64_t)((sl * kBox + 2 * blk * kKbStride + ks * 2048) >> 4);
+                                        const uint64_t bd =
+                                            dp0 + (uint64_t)((pb * kPBuf + j * kPTerm + g * 4096 + ks * 32) >> 4);
+                                        umma::mma_f8(t_o + blk * HQ, ad, bd, IDESC_PV,
+                                                     (fst && j == 0 && g == 0 && ks == 0) ? 0u : 1u);
+                                    }
+                            umma::commit(bar + B_PAGE_EMPTY + sl);
+                        }
                         umma::commit(bar + B_PV_DONE + pb);
-                        umma::commit(bar + B_TILE_EMPTY + st);
+                        TRACE(4, next_pv);
                         next_pv++;
                         progress = true;
                     }
                 }
-                if (!sentinel && next_s - next_pv < 2) {
-                    const int st = next_s % kStages;
-                    if (mbar_test(bar + B_TILE_FULL + st, (next_s / kStages) & 1)) {
-                        const StageMeta meta = load_meta(tmeta + st);
+                // S(k) needs its two pages, the S columns read out by the softmax (tile k-1)
+                // and the query rows of its unit
+                if (!sentinel && next_s - next_pv < 2 &&
+                    (next_s == 0 || mbar_test(bar + B_S_FREE, (next_s - 1) & 1))) {
+                    const uint32_t p0 = 2 * next_s, p1 = p0 + 1;
+                    const int s0 = slot_of(p0), s1 = slot_of(p1);
+                    if (mbar_test(bar + B_PAGE_FULL + s0, phase_of(p0))) {
+                        const StageMeta meta = load_meta(tmeta + s0);
                         if (meta.unit < 0) {
                             sentinel = true;
-                        } else {
+                        } else if (mbar_test(bar + B_PAGE_FULL + s1, phase_of(p1))) {
                             const bool first = meta.flags & kStageFirst;
                             if (!first || mbar_test(bar + B_Q_FULL, unit_k & 1)) {
                                 if (first) unit_k++;
+                                TRACE(0, next_s);
                                 umma::fence_after_sync();
-                                const int sb = next_s & 1;
-                                const uint64_t tile = (uint64_t)((st * kTileBytes) >> 4);
+                                if (s1 == s0 + 1) {
+                                    // adjacent slots: one 128-row operand
+                                    const uint32_t tile = (uint32_t)(s0 * kBox);
 #pragma unroll
-                                for (int kb = 0; kb < kKB; kb++)
+                                    for (int kb = 0; kb < 8; kb++)
 #pragma unroll
-                                    for (int ks = 0; ks < 2; ks++) {
-                                        const uint64_t aq = dq0 + (uint64_t)((kb * kQBox + ks * 32) >> 4);
-                                        const uint64_t bt = dt0 + tile + (uint64_t)((kb * kBox + ks * 32) >> 4);
-                                        umma::mma_f8(t_s + sb * kT, aq, bt, IDESC_S, (kb | ks) ? 1u : 0u);
+                                        for (int ks = 0; ks < 2; ks++)
+                                            umma::mma_f8_ts(t_s, t_q + (2 * kb + ks) * 8,
+                                                            dt0 + (uint64_t)((tile + kb * kKbStride + ks * 32) >> 4),
+                                                            IDESC_S128, (kb | ks) ? 1u : 0u);
+#pragma unroll
+                                    for (int ks = 0; ks < 2; ks++)
+                                        umma::mma_f8(t_s, dr0 + (uint64_t)((ks * 32) >> 4),
+                                                     dt0 + (uint64_t)((tile + 8 * kKbStride + ks * 32) >> 4),
+                                                     IDESC_S128, 1u);
+                                } else {
+                                    // the ring wraps between the two pages: two 64-row halves
+#pragma unroll
+                                    for (int g = 0; g < 2; g++) {
+                                        const uint32_t tile = (uint32_t)((g ? s1 : s0) * kBox);
+#pragma unroll
+                                        for (int kb = 0; kb < 8; kb++)
+#pragma unroll
+                                            for (int ks = 0; ks < 2; ks++)
+                                                umma::mma_f8_ts(t_s + 64 * g, t_q + (2 * kb + ks) * 8,
+                                                                dt0 + (uint64_t)((tile + kb * kKbStride + ks * 32) >> 4),
+                                                                IDESC_S64, (kb | ks) ? 1u : 0u);
+#pragma unroll
+                                        for (int ks = 0; ks < 2; ks++)
+                                            umma::mma_f8(t_s + 64 * g, dr0 + (uint64_t)((ks * 32) >> 4),
+                                                         dt0 + (uint64_t)((tile + 8 * kKbStride + ks * 32) >> 4),
+                                                         IDESC_S64, 1u);
                                     }
-                                umma::commit(bar + B_S_FULL + sb);
+                                }
+                                umma::commit(bar + B_S_FULL);
                                 if (meta.flags & kStageLast) umma::commit(bar + B_Q_FREE);
-                                first_bits = (first_bits & ~(1u << sb)) | ((first ? 1u : 0u) << sb);
+                                TRACE(1, next_s);
+                                const int ts = next_s & 1;
+                                first_bits = (first_bits & ~(1u << ts)) | ((first ? 1u : 0u) << ts);
                                 next_s++;
                                 progress = true;
                             }
@@ -305,6 +481,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (progress) {
                     t_prog = global_timer_ns();
                 } else {
+                    // nothing ready: yield the issue slots this warp shares with softmax warps
+                    __nanosleep(32);
                     if (*s_abort) break;
                     if (global_timer_ns() - t_prog > kWaitLimitNs) {
                         record_status(a.status, DCP_ERR_TIMEOUT);
@@ -317,90 +495,69 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_wait(bar + B_FINAL, 0, nullptr, a.status);
         }
     } else {
-        // ------------------------------------------------------------------ q split, softmax, epilogue
-        const int qd = warp & 3;                    // TMEM lane quadrant
-        const int h = 32 * (qd & 1) + lane;         // head
-        const int half = qd >> 1;                   // 0: holds S_hi, finishes tokens 0..31; 1: S_lo, tokens 32..63
+        // ------------------------------------------------------------------ query rows, softmax, epilogue
+        const int qd = warp & 3;                  // TMEM lane quadrant
+        const int wg = (warp - 2) >> 2;           // token group: tile tokens 64 wg .. 64 wg + 63 (page wg)
+        const int half = lane >> 4;               // 0: row holds S_hi; 1: S_lo
+        const int h = 16 * qd + (lane & 15);      // head
         const bool head = h < HQ;
-        const int tid = threadIdx.x - 64;           // 0..127
-        const int sw = warp - 2;                    // 0..3
+        const int row = 32 * qd + lane;           // query row = TMEM lane
+        const int base = 64 * wg + 32 * half;     // my 32 tokens of the tile
+        const int tid = threadIdx.x - 64;         // 0..255
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
         uint32_t seq = 0, unit_k = 0;
-        float m_used = -INFINITY, lpart = 0.f;
+        float m_used = -INFINITY, lpart = 0.f, f = 0.f;
         bool o_has = false, fail = false;
         Unit u;
         u.n = u.b = u.t0 = u.t1 = u.slot = u.n_chunks = u.slot_base = u.pad = 0;
-        float* xrow_out = xbuf + ((size_t)half * 64 + h) * 32;        // my half of the exchange
-        const float* xrow_in = xbuf + ((size_t)(half ^ 1) * 64 + h) * 32;
         while (true) {
-            const int st = seq % kStages;
-            const int sb = seq & 1;
-            if (!fail) fail = !mbar_wait(bar + B_TILE_FULL + st, (seq / kStages) & 1, s_abort, a.status);
+            const int ts = seq & 1;
+            const int s0 = slot_of(2 * seq), s1 = slot_of(2 * seq + 1);
+            if (!fail) fail = !mbar_wait(bar + B_PAGE_FULL + s0, phase_of(2 * seq), s_abort, a.status);
             StageMeta meta{-1, 0, 0, 0};
-            if (!fail) meta = load_meta(tmeta + st);
-            if (named_barrier_or(kSmBar, 128, fail)) break;
+            if (!fail) meta = load_meta(tmeta + s0);
+            if (named_barrier_or(kSmBar, 256, fail)) break;
             if (meta.unit < 0) break;
             const bool first = meta.flags & kStageFirst;
             const bool last = meta.flags & kStageLast;
             const int nvalid = (meta.flags >> 8) & 0xFF;
+            const bool full = nvalid == kT;
+            const int my_slot = wg ? s1 : s0;  // page holding my tokens
             if (first) {
                 u = a.units[meta.unit];
+                f = head ? __ldg(a.qinv + (int64_t)u.b * 64 + h) * a.scale_log2 : 0.f;
                 // the previous unit's S MMAs are complete (first unit passes at once)
                 fail = !mbar_wait(bar + B_Q_FREE, (unit_k & 1) ^ 1, s_abort, a.status);
                 if (!fail) {
-                    // warp sw splits heads sw*16 .. sw*16+15 of request u.b; lane c handles
-                    // 16-element chunk c (and c + 32 for c < 4) of the 576-wide row
-                    for (int hh = sw * 16; hh < sw * 16 + 16 && hh < HQ; hh++) {
-                        const uint4* qrow = reinterpret_cast<const uint4*>(a.q + ((int64_t)u.b * HQ + hh) * 576);
-                        uint4 w[2][2];
-                        float amax = 0.f;
+                    if (head) {
+                        // token group wg copies query bytes [256 wg, 256 wg + 256) -> TMEM columns 64 wg ..
+                        const uint4* src = reinterpret_cast<const uint4*>(a.qs + ((int64_t)u.b * 128 + row) * 576);
+                        uint4 v[16];
 #pragma unroll
-                        for (int k2 = 0; k2 < 2; k2++) {
-                            const int c = lane + 32 * k2;
-                            if (c < 36) {
-                                w[k2][0] = __ldg(qrow + 2 * c);
-                                w[k2][1] = __ldg(qrow + 2 * c + 1);
-                                const uint32_t ws[8] = {w[k2][0].x, w[k2][0].y, w[k2][0].z, w[k2][0].w,
-                                                        w[k2][1].x, w[k2][1].y, w[k2][1].z, w[k2][1].w};
+                        for (int i = 0; i < 16; i++) v[i] = __ldg(src + 16 * wg + i);
+                        uint32_t r0[32], r1[32];
 #pragma unroll
-                                for (int e = 0; e < 8; e++)
-                                    amax = fmaxf(amax, fmaxf(fabsf(bf16_lo(ws[e])), fabsf(bf16_hi(ws[e]))));
-                            }
+                        for (int i = 0; i < 8; i++) {
+                            r0[4 * i] = v[i].x;
+                            r0[4 * i + 1] = v[i].y;
+                            r0[4 * i + 2] = v[i].z;
+                            r0[4 * i + 3] = v[i].w;
+                            r1[4 * i] = v[8 + i].x;
+                            r1[4 * i + 1] = v[8 + i].y;
+                            r1[4 * i + 2] = v[8 + i].z;
+                            r1[4 * i + 3] = v[8 + i].w;
                         }
+                        umma::st32(t_q + lane_off + 64 * wg, r0);
+                        umma::st32(t_q + lane_off + 64 * wg + 32, r1);
+                        if (wg == 1) {
 #pragma unroll
-                        for (int o = 16; o; o >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, o));
-                        int ex = 0;
-                        frexpf(amax, &ex);                       // amax in [2^(ex-1), 2^ex)
-                        ex = max(ex, -110);                       // sigma and 1/sigma stay finite
-                        const float sig = amax > 0.f ? ldexpf(1.f, 8 - ex) : 1.f;
-                        if (lane == 0) s_qs[hh] = 1.f / sig;
-#pragma unroll
-                        for (int k2 = 0; k2 < 2; k2++) {
-                            const int c = lane + 32 * k2;
-                            if (c < 36) {
-                                const uint32_t ws[8] = {w[k2][0].x, w[k2][0].y, w[k2][0].z, w[k2][0].w,
-                                                        w[k2][1].x, w[k2][1].y, w[k2][1].z, w[k2][1].w};
-                                uint32_t hi[4], lo[4];
-#pragma unroll
-                                for (int e = 0; e < 4; e++) {
-                                    const float a0 = bf16_lo(ws[2 * e]) * sig, a1 = bf16_hi(ws[2 * e]) * sig;
-                                    const float a2 = bf16_lo(ws[2 * e + 1]) * sig, a3 = bf16_hi(ws[2 * e + 1]) * sig;
-                                    const uint32_t h01 = to_e4m3x2(a0, a1), h23 = to_e4m3x2(a2, a3);
-                                    const float2 d01 = from_fp8x2(h01, __NV_E4M3), d23 = from_fp8x2(h23, __NV_E4M3);
-                                    const uint32_t l01 = to_e4m3x2(a0 - d01.x, a1 - d01.y);
-                                    const uint32_t l23 = to_e4m3x2(a2 - d23.x, a3 - d23.y);
-                                    hi[e] = h01 | (h23 << 16);
-                                    lo[e] = l01 | (l23 << 16);
-                                }
-                                // chunk c: bytes [16c, 16c+16) of the row = box c/4, 16-byte chunk c%4
-                                uint8_t* qb = sm + kOffQ + (c >> 2) * kQBox;
-                                *reinterpret_cast<uint4*>(qb + sw64(hh, c & 3)) = make_uint4(hi[0], hi[1], hi[2], hi[3]);
-                                *reinterpret_cast<uint4*>(qb + sw64(64 + hh, c & 3)) =
-                                    make_uint4(lo[0], lo[1], lo[2], lo[3]);
-                            }
+                            for (int c = 0; c < 4; c++)
+                                *reinterpret_cast<uint4*>(sm + kOffRope + sw64(row, c)) = __ldg(src + 32 + c);
                         }
                     }
+                    umma::wait_st();
                     umma::fence_proxy_async_smem();
+                    umma::fence_before_sync();
                     __syncwarp();
                     if (lane == 0) mbar_arrive(bar + B_Q_FULL);
                 }
@@ -409,66 +566,89 @@ __global__ void __launch_bounds__(kThreads, 1)
                 lpart = 0.f;
                 o_has = false;
             }
-            // ---- scores: S_hi / S_lo rows, exchange halves
-            if (!fail) fail = !mbar_wait(bar + B_S_FULL + sb, (seq >> 1) & 1, s_abort, a.status);
+            // ---- scores: rows S_hi (lane < 16) and S_lo (lane >= 16) of head h; swap halves
+            if (!fail) fail = !mbar_wait(bar + B_S_FULL, seq & 1, s_abort, a.status);
             umma::fence_after_sync();
-            uint32_t mine[32], other[32];
-            umma::ld32(t_s + lane_off + sb * kT, mine);
-            umma::ld32(t_s + lane_off + sb * kT + 32, other);
-            umma::wait_ld();
-            // half 0 keeps tokens 0..31 and sends 32..63; half 1 the reverse
-#pragma unroll
-            for (int j = 0; j < 32; j++) {
-                const uint32_t m0 = half ? other[j] : mine[j], o0 = half ? mine[j] : other[j];
-                mine[j] = m0;
-                other[j] = o0;
-            }
-#pragma unroll
-            for (int c = 0; c < 8; c++)   // rotated 16-byte chunks: no bank conflicts
-                *reinterpret_cast<uint4*>(xrow_out + (((c + h) & 7) << 2)) =
-                    make_uint4(other[4 * c], other[4 * c + 1], other[4 * c + 2], other[4 * c + 3]);
-            named_barrier_sync(kSmBar, 128);
-            const int base = half ? 32 : 0;  // my tokens
+            if (threadIdx.x == 64) TRACE(5, seq);
+            const float4* tsc4 = reinterpret_cast<const float4*>(sm + kOffScales + my_slot * kPg * 4 + 32 * half * 4);
             float x[32];
+            float smax = 0.f;
             {
-                const float* tsc = reinterpret_cast<const float*>(sm + kOffScales + st * kT * 4) + base;
-                const float f = head ? s_qs[h] * a.scale_log2 : 0.f;
+                uint32_t v0[32], v1[32];
+                umma::ld32(t_s + lane_off + 64 * wg, v0);
+                umma::ld32(t_s + lane_off + 64 * wg + 32, v1);
+                umma::wait_ld();
+                // the S columns may be overwritten by the next tile's MMAs from here on
+                umma::fence_before_sync();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(bar + B_S_FREE);
 #pragma unroll
-                for (int c = 0; c < 8; c++) {
-                    const float4 o4 = *reinterpret_cast<const float4*>(xrow_in + (((c + h) & 7) << 2));
-                    const float ov[4] = {o4.x, o4.y, o4.z, o4.w};
+                for (int j4 = 0; j4 < 8; j4++) {
+                    const float4 sc4 = tsc4[j4];
+                    const float sc[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
-                        const int j = 4 * c + e;
-                        const float s = __uint_as_float(mine[j]) + ov[e];
-                        x[j] = (base + j < nvalid) ? s * f * tsc[j] : -INFINITY;
+                        const int j = 4 * j4 + e;
+                        const uint32_t keep = half ? v1[j] : v0[j], send = half ? v0[j] : v1[j];
+                        const float s =
+                            __uint_as_float(keep) + __uint_as_float(__shfl_xor_sync(0xffffffffu, send, 16));
+                        x[j] = s * f * sc[e];
+                        smax = fmaxf(smax, sc[e]);
+                    }
+                }
+                if (!full) {
+                    // tokens past the end of the unit: no score, and their stale scales do not count
+                    smax = 0.f;
+#pragma unroll
+                    for (int j4 = 0; j4 < 8; j4++) {
+                        const float4 sc4 = tsc4[j4];
+                        const float sc[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
+#pragma unroll
+                        for (int e = 0; e < 4; e++) {
+                            const bool valid = base + 4 * j4 + e < nvalid;
+                            x[4 * j4 + e] = valid ? x[4 * j4 + e] : -INFINITY;
+                            smax = valid ? fmaxf(smax, sc[e]) : smax;
+                        }
                     }
                 }
             }
-            float mt = -INFINITY;
+            if (threadIdx.x == 64) TRACE(6, seq);
+            float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 32; j++) mt = fmaxf(mt, x[j]);
-            xmax[half * 64 + h] = mt;
-            named_barrier_sync(kSmBar, 128);
-            mt = fmaxf(mt, xmax[(half ^ 1) * 64 + h]);
+            for (int j = 0; j < 32; j++) mx = fmaxf(mx, x[j]);
+            mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
+            smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
+            // combine with the other token group of the same heads
+            if (half == 0) {
+                s_gmax[wg * 64 + h] = mx;
+                s_gsmax[wg * 64 + h] = smax;
+            }
+            named_barrier_sync(kPairBar + qd, 64);
+            mx = fmaxf(mx, s_gmax[(wg ^ 1) * 64 + h]);
+            smax = fmaxf(smax, s_gsmax[(wg ^ 1) * 64 + h]);
+            // m >= max_t (x_t + log2 s_t): the weights 2^(x - m) s_t stay <= 2^8
+            const float mt = (mx == -INFINITY || !(smax > 0.f)) ? mx : mx + __log2f(smax);
             float alpha = 1.f;
             if (mt > m_used + kRescaleLog2 || (m_used == -INFINITY && mt != -INFINITY)) {
                 alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - mt);
                 m_used = mt;
             }
-            if (half == 0) s_alpha[h] = alpha;
+            if (half == 0 && wg == 0) s_alpha[h] = alpha;
+            if (threadIdx.x == 64) TRACE(7, seq);
             // one barrier: some head rescaled while O^T holds data, or a wait failed (a failing
             // thread republishes the abort flag first, so every thread reads it set after the barrier)
             if (fail) *s_abort = 1;
-            const int any = named_barrier_or(kSmBar, 128, fail || (head && alpha != 1.f && o_has));
+            const int any = named_barrier_or(kSmBar, 256, fail || (head && alpha != 1.f && o_has));
             if (any && *s_abort) break;
+            if (threadIdx.x == 64) TRACE(8, seq);
             if (any) {
-                // the previous tile's P V must be complete before O^T is rescaled
-                fail = !mbar_wait(bar + B_PV_DONE + (sb ^ 1), ((seq - 1) >> 1) & 1, s_abort, a.status);
+                // the previous tile's P V must be complete before O^T is rescaled; token group wg
+                // rescales value blocks 2 wg, 2 wg + 1 of its lane quadrant
+                fail = !mbar_wait(bar + B_PV_DONE + (ts ^ 1), ((seq - 1) >> 1) & 1, s_abort, a.status);
                 if (!fail) {
                     umma::fence_after_sync();
 #pragma unroll 1
-                    for (int blk = 0; blk < 4; blk++) {
+                    for (int blk = 2 * wg; blk < 2 * wg + 2; blk++) {
 #pragma unroll 1
                         for (int c0 = 0; c0 < HQ; c0 += 16) {
                             uint32_t r[16];
@@ -483,115 +663,118 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma::wait_st();
                 }
             }
-            // ---- P' = 16 p s_t as three e5m2 terms (the P buffer is free once P V of tile seq-2 is done)
-            if (!fail) fail = !mbar_wait(bar + B_PV_DONE + sb, ((seq >> 1) & 1) ^ 1, s_abort, a.status);
+            // ---- W = p s_t as two e4m3 terms (the P buffer is free once P V of tile seq-2 is done)
+            if (!fail) fail = !mbar_wait(bar + B_PV_DONE + ts, ((seq >> 1) & 1) ^ 1, s_abort, a.status);
+            if (threadIdx.x == 64) TRACE(10, seq);
             if (!fail && head) {
-                const float* tsc = reinterpret_cast<const float*>(sm + kOffScales + st * kT * 4) + base;
+                float w[32];
                 float rowsum = 0.f;
-                uint32_t t0[8], t1[8], t2[8];
+                if (m_used != -INFINITY) {
+                    // 2^(-inf - m) = 0 for masked tokens; stale scales are zeroed below
 #pragma unroll
-                for (int j = 0; j < 32; j += 4) {
-                    float pp[4];
+                    for (int j4 = 0; j4 < 8; j4++) {
+                        const float4 sc4 = tsc4[j4];
+                        const float sc[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
 #pragma unroll
-                    for (int e = 0; e < 4; e++) {
-                        const float p = x[j + e] == -INFINITY ? 0.f : fast_exp2(x[j + e] - m_used);
-                        rowsum += p;
-                        pp[e] = p > 0.f ? p * tsc[j + e] * kPScale : 0.f;  // stale scales meet no p = 0
+                        for (int e = 0; e < 4; e++) {
+                            const float p = fast_exp2(x[4 * j4 + e] - m_used);
+                            rowsum += p;
+                            w[4 * j4 + e] = p * sc[e];
+                        }
                     }
-                    uint32_t c0[2], c1[2], c2[2];
+                    if (!full) {
 #pragma unroll
-                    for (int e = 0; e < 2; e++) {
-                        const float a0 = pp[2 * e], a1 = pp[2 * e + 1];
-                        c0[e] = to_e5m2x2(a0, a1);
-                        const float2 d0 = from_fp8x2(c0[e], __NV_E5M2);
-                        const float r0 = a0 - d0.x, r1 = a1 - d0.y;
-                        c1[e] = to_e5m2x2(r0, r1);
-                        const float2 d1 = from_fp8x2(c1[e], __NV_E5M2);
-                        c2[e] = to_e5m2x2(r0 - d1.x, r1 - d1.y);
+                        for (int j = 0; j < 32; j++) w[j] = (base + j < nvalid) ? w[j] : 0.f;
                     }
-                    t0[j / 4] = c0[0] | (c0[1] << 16);
-                    t1[j / 4] = c1[0] | (c1[1] << 16);
-                    t2[j / 4] = c2[0] | (c2[1] << 16);
+                } else {
+#pragma unroll
+                    for (int j = 0; j < 32; j++) w[j] = 0.f;
                 }
+                uint32_t chi[8], clo[8];
+                split32(w, chi, clo);
                 lpart = lpart * alpha + rowsum;
-                uint8_t* pb = sm + kOffP + sb * kPBuf;
-                // my 32 tokens = 16-byte chunks 2*half and 2*half + 1 of row h
+                // page wg of the tile, row h, 16-byte chunks 2 half and 2 half + 1
+                uint8_t* pb = sm + kOffP + ts * kPBuf + wg * 4096;
 #pragma unroll
                 for (int cc = 0; cc < 2; cc++) {
                     const int c = 2 * half + cc;
-                    *reinterpret_cast<uint4*>(pb + 0 * kPTerm + sw64(h, c)) =
-                        make_uint4(t0[4 * cc], t0[4 * cc + 1], t0[4 * cc + 2], t0[4 * cc + 3]);
-                    *reinterpret_cast<uint4*>(pb + 1 * kPTerm + sw64(h, c)) =
-                        make_uint4(t1[4 * cc], t1[4 * cc + 1], t1[4 * cc + 2], t1[4 * cc + 3]);
-                    *reinterpret_cast<uint4*>(pb + 2 * kPTerm + sw64(h, c)) =
-                        make_uint4(t2[4 * cc], t2[4 * cc + 1], t2[4 * cc + 2], t2[4 * cc + 3]);
+                    *reinterpret_cast<uint4*>(pb + sw64(h, c)) =
+                        make_uint4(chi[4 * cc], chi[4 * cc + 1], chi[4 * cc + 2], chi[4 * cc + 3]);
+                    *reinterpret_cast<uint4*>(pb + kPTerm + sw64(h, c)) =
+                        make_uint4(clo[4 * cc], clo[4 * cc + 1], clo[4 * cc + 2], clo[4 * cc + 3]);
                 }
             } else if (!fail) {
                 lpart = lpart * alpha;
             }
-            if (!fail && nvalid < kT) {
+            if (!fail && !full) {
                 // rows past the last valid token hold stale page bytes (possibly NaN codes):
-                // zero their value columns so that P = 0 cannot meet them
-                uint8_t* tile = sm + kOffTiles + (size_t)st * kTileBytes;
+                // zero their value columns so that W = 0 cannot meet them
                 const int nr = kT - nvalid;
-                for (int i = tid; i < nr * 4 * 8; i += 128) {
-                    const int box = i / (nr * 4), rem = i - box * nr * 4;
-                    const int r = nvalid + rem / 4, c = rem & 3;
-                    *reinterpret_cast<uint4*>(tile + box * kBox + r * 64 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+                for (int i = tid; i < nr * 4 * 8; i += 256) {
+                    const int kb = i / (nr * 4), rem = i - kb * nr * 4;
+                    const int tok = nvalid + rem / 4, c = rem & 3;
+                    *reinterpret_cast<uint4*>(sm + kOffTiles + kb * kKbStride + (tok < kPg ? s0 : s1) * kBox +
+                                              (tok % kPg) * 64 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
             umma::fence_proxy_async_smem();
             umma::fence_before_sync();
             __syncwarp();
-            if (!fail && lane == 0) mbar_arrive(bar + B_P_FULL + sb);
+            if (!fail && lane == 0) mbar_arrive(bar + B_P_FULL + ts);
+            if (threadIdx.x == 64) TRACE(9, seq);
             o_has = true;
-            // ---- end of unit: O = O^T / (16 l), LSE
+            // ---- end of unit: O = O^T / l, LSE
             if (last) {
-                if (!fail) fail = !mbar_wait(bar + B_PV_DONE + sb, (seq >> 1) & 1, s_abort, a.status);
+                if (threadIdx.x == 64) TRACE(12, seq);
+                if (!fail) fail = !mbar_wait(bar + B_PV_DONE + ts, (seq >> 1) & 1, s_abort, a.status);
                 umma::fence_after_sync();
-                (half ? s_l1 : s_l0)[h] = lpart;
-                if (half == 0) s_m[h] = m_used;
-                if (named_barrier_or(kSmBar, 128, fail)) break;
+                const float lg = lpart + __shfl_xor_sync(0xffffffffu, lpart, 16);  // this token group
+                if (half == 0) s_gl[wg * 64 + h] = lg;
                 const int64_t shard = (int64_t)u.n * a.batch + u.b;
                 const bool split = u.n_chunks > 1;
                 float* obase = split ? a.split_o + (int64_t)u.slot * a.hq * 512 : a.o_partial + shard * a.hq * 512;
                 float* lbase = split ? a.split_lse + (int64_t)u.slot * a.hq : a.lse + shard * a.hq;
+                if (named_barrier_or(kSmBar, 256, fail)) break;
+                if (head && half == 0 && wg == 0) {
+                    const float l = lg + s_gl[64 + h];
+                    s_inv[h] = l > 0.f ? 1.f / l : 0.f;
+                    __stcg(lbase + h, l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY);
+                }
+                named_barrier_sync(kSmBar, 256);
 #pragma unroll 1
-                for (int blk = 0; blk < 4; blk++) {
-                    const int dv = blk * 128 + 32 * qd + lane;
+                for (int c0 = 0; c0 < HQ; c0 += 16) {
+                    float inv[16];
+#pragma unroll
+                    for (int i = 0; i < 16; i++) inv[i] = s_inv[c0 + i];
 #pragma unroll 1
-                    for (int c0 = 0; c0 < HQ; c0 += 16) {
+                    for (int blk = 2 * wg; blk < 2 * wg + 2; blk++) {
+                        const int dv = blk * 128 + 32 * qd + lane;
                         uint32_t r[16];
                         umma::ld16(t_o + lane_off + blk * HQ + c0, r);
                         umma::wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 16; i++) {
-                            const float l = s_l0[c0 + i] + s_l1[c0 + i];
-                            __stcg(obase + (int64_t)(c0 + i) * 512 + dv,
-                                   l > 0.f ? __uint_as_float(r[i]) / (kPScale * l) : 0.f);
-                        }
+                        for (int i = 0; i < 16; i++)
+                            __stcg(obase + (int64_t)(c0 + i) * 512 + dv, __uint_as_float(r[i]) * inv[i]);
                     }
-                }
-                if (half == 0 && head) {
-                    const float l = s_l0[h] + s_l1[h];
-                    __stcg(lbase + h, l > 0.f ? (s_m[h] + log2f(l)) * kLn2 : -INFINITY);
                 }
                 umma::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar + B_O_FREE);
                 if (split) {
                     __threadfence();
-                    named_barrier_sync(kSmBar, 128);
+                    named_barrier_sync(kSmBar, 256);
                     if (tid == 0) s_misc[2] = (atomicAdd(a.done + shard, 1) == u.n_chunks - 1) ? 1 : 0;
-                    named_barrier_sync(kSmBar, 128);
+                    named_barrier_sync(kSmBar, 256);
                     const int is_last = *reinterpret_cast<volatile int*>(s_misc + 2);
-                    named_barrier_sync(kSmBar, 128);
+                    named_barrier_sync(kSmBar, 256);
                     if (is_last) {
                         __threadfence();
-                        merge_split_chunks(a, u, shard, 0, HQ, tid, 128);
+                        merge_split_chunks(a, u, shard, 0, HQ, tid, 256);
                     }
                 }
+                if (threadIdx.x == 64) TRACE(13, seq);
             }
+            if (threadIdx.x == 64) TRACE(11, seq);
             seq++;
         }
     }
@@ -608,10 +791,14 @@ template <int HQ>
 cudaError_t run(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s) {
     CUtensorMap tm;
     if (!make_tmap_2d(&tm, a.k_pages, CU_TENSOR_MAP_DATA_TYPE_UINT8, 576, (uint64_t)a.num_pages * a.page_size, 576, 64,
-                      kT, CU_TENSOR_MAP_SWIZZLE_64B))
+                      kPg, CU_TENSOR_MAP_SWIZZLE_64B))
         return cudaErrorInvalidValue;
+    const int warps = a.batch * HQ;
+    mla_fp8_qsplit_kernel<<<(warps + 3) / 4, 128, 0, s>>>(a.q, a.batch, HQ, a.qs, a.qinv);
+    cudaError_t e = cudaGetLastError();
+    if (e != cudaSuccess) return e;
     auto fn = mla_fp8_kernel<HQ>;
-    cudaError_t e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
+    e = cudaFuncSetAttribute(fn, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)kSmemBytes);
     if (e != cudaSuccess) return e;
     fn<<<g.ctas, kThreads, kSmemBytes, s>>>(tm, a);
     return cudaGetLastError();
@@ -620,6 +807,7 @@ cudaError_t run(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s) {
 }  // namespace
 
 cudaError_t launch_decode_mla_fp8(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s) {
+    if (!a.qs || !a.qinv) return cudaErrorInvalidValue;
     switch (a.hq) {
         case 16: return run<16>(g, a, s);
         case 32: return run<32>(g, a, s);
