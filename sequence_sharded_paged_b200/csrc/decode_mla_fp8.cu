@@ -18,33 +18,34 @@
 // in one warp's TMEM lane quadrant.  The first 512 columns of those rows live
 // in tensor memory (the MMA's A operand), the 64 rope columns in shared memory.
 //
-// Scores.  [S_hi; S_lo] = [Q_hi; Q_lo] . C^T, M = 128, N = 128 tokens, K = 576:
-// 16 MMAs with A in TMEM + 2 with A in shared memory; the two pages of the tile
-// are the only shared-memory operand.  Lane pairs (l, l + 16) swap halves with
-// shuffles and form s = scale * s_t * (S_hi + S_lo) / sigma_h.
+// Scores.  [S_hi; S_lo] = [Q_hi; Q_lo] . C^T per page, M = 128, N = 64 tokens,
+// K = 576: 16 MMAs with A in TMEM + 2 with A in shared memory; the page is the
+// only shared-memory operand.  Lane pairs (l, l + 16) swap halves with shuffles
+// and form s = scale * s_t * (S_hi + S_lo) / sigma_h.
 //
-// Values.  O^T = V^T . W^T with V^T read MN-major straight from the raw pages
+// Values.  O^T = V^T . W^T with V^T read MN-major straight from the raw page
 // and W = p * s_t in two e4m3 terms (relative error below 2^-8).  The running
-// maximum m absorbs the tile's largest scale (m >= max_t (x_t + log2 s_t), x in
+// maximum m absorbs the page's largest scale (m >= max_t (x_t + log2 s_t), x in
 // log2 units), so W = 2^(x - m) s_t <= 2^8 stays inside e4m3's range whatever
 // the scales; it is rescaled lazily (O^T only when m grows by more than 2^8).
-//   O^T += V^T . W_j^T   M = 128 value columns (4 blocks), N = Hq, K = 128, j = 0, 1
-// 32 MMAs per tile.  O = O^T / l with l = sum_t 2^(x_t - m).
+//   O^T += V^T . W_j^T   M = 128 value columns (4 blocks), N = Hq, K = 64, j = 0, 1
+// 16 MMAs per page.  O = O^T / l with l = sum_t 2^(x_t - m).
 //
-// Tiles: two 64-token pages (128 tokens).  Each page arrives as nine
-// [64 rows][64 B] TMA boxes with 64-byte swizzle (36 KB) + 256 B of scales;
-// block kb of the four page slots is contiguous, so that the two pages of a
-// tile form one 128-row operand.  Two tiles in flight.
+// Pages: nine [64 rows][64 B] TMA boxes with 64-byte swizzle (36 KB) + 256 B
+// of scales, in a ring of five slots; a slot is refilled as soon as P V of its
+// page completes.
 //
 // Warp roles (one CTA per SM, persistent, units from an atomic ticket):
-//   warp 0      TMA producer (lane 0)
-//   warp 1      TMEM allocation, MMA issue (lane 0, event loop)
+//   warp 0      producer: tickets, page indices (one page of lookahead), TMA
+//   warp 1      TMEM allocation; issues the scores of each page
 //   warps 2..9  query rows, softmax, lazy rescale of O^T, epilogue.  The two
 //               warps on TMEM quadrant j own heads 16 j .. 16 j + 15: warp
-//               group g (warps 2..5: g = 0, 6..9: g = 1) the tile's tokens
-//               64 g .. 64 g + 63, in which lane l < 16 takes the first 32
-//               and lane l + 16 the last 32; g also picks the value blocks
+//               group g (warps 2..5: g = 0, 6..9: g = 1) the page's tokens
+//               32 g .. 32 g + 31, in which lane l < 16 takes the first 16
+//               and lane l + 16 the last 16; g also picks the value blocks
 //               2 g, 2 g + 1 that the warp rescales and stores.
+//   warp 10     issues P V of each page
+// Scores run up to two pages ahead of the softmax (two S buffers in TMEM).
 #include "common.cuh"
 #include "finish.cuh"
 #include "kernels.h"
@@ -56,7 +57,7 @@ namespace dcp {
 // Optional timeline of CTA 0 (SM clock at each protocol step), compiled only
 // with -DDCP_TRACE for profiling builds; expands to nothing otherwise.
 #ifdef DCP_TRACE
-__device__ unsigned long long g_mla8_trace[16][512];
+__device__ unsigned long long g_mla8_trace[40][512];
 #define TRACE(ev, k)                                                          \
     do {                                                                      \
         if (blockIdx.x == 0 && (k) < 512) g_mla8_trace[ev][(k)] = clock64();  \
@@ -72,25 +73,23 @@ extern "C" int dcp_trace8_read(unsigned long long* host) {
 
 namespace {
 
-constexpr int kPg = 64;                    // tokens per page
-constexpr int kT = 128;                    // tokens per tile (two pages)
+constexpr int kPg = 64;                    // tokens per page = tokens per tile
 constexpr int kKB = 9;                     // 576 = 9 blocks of 64 bytes
-constexpr int kBox = kPg * 64;             // [64 rows][64 B] box of one page: 4 KB
-constexpr int kSlots = 5;                  // page slots: two and a half tiles in flight
-constexpr int kKbStride = kSlots * kBox;   // block kb of every slot: [slot][64 rows][64 B]
-constexpr int kPageBytes = kKB * kBox;     // 36864
+constexpr int kBox = kPg * 64;             // [64 rows][64 B] box: 4 KB
+constexpr int kTileBytes = kKB * kBox;     // one page: 36864
+constexpr int kSlots = 5;                  // pages in flight
 constexpr int kRopeBytes = 128 * 64;       // rope columns of the 128 query rows
-constexpr int kPTerm = 64 * 128;           // W_j^T [2 pages][64 heads][64 tokens] e4m3: 8 KB
-constexpr int kPBuf = 2 * kPTerm;          // 16 KB
+constexpr int kPTerm = 64 * 64;            // W_j^T [64 heads][64 tokens] e4m3: 4 KB
+constexpr int kPBuf = 2 * kPTerm;          // 8 KB
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kSmBar = 1;                  // the 256 softmax threads
 constexpr int kPairBar = 2;                // + quadrant: the two warps sharing a TMEM lane quadrant
 constexpr int kSoftWarps = 8;
-constexpr int kThreads = 32 * (2 + kSoftWarps);
+constexpr int kThreads = 32 * (3 + kSoftWarps);  // producer, S issuer, softmax x 8, P V issuer
 constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384;  // TMEM columns
 
 constexpr uint32_t kOffTiles = 0;
-constexpr uint32_t kOffRope = kOffTiles + kKB * kKbStride;
+constexpr uint32_t kOffRope = kOffTiles + kSlots * kTileBytes;
 constexpr uint32_t kOffP = kOffRope + kRopeBytes;
 constexpr uint32_t kOffScales = kOffP + 2 * kPBuf;
 constexpr uint32_t kOffBars = kOffScales + kSlots * kPg * 4;
@@ -104,21 +103,20 @@ static_assert(kOffRope % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands need
 enum : int {
     B_PAGE_FULL = 0,    // [kSlots]
     B_PAGE_EMPTY = 8,   // [kSlots]
-    B_S_FULL = 16,
-    B_S_FREE = 17,
-    B_P_FULL = 18,      // [2]
-    B_PV_DONE = 20,     // [2]
-    B_Q_FULL = 22,
-    B_Q_FREE = 23,
-    B_O_FREE = 24,
-    B_FINAL = 25,
+    B_S_FULL = 16,      // [2]
+    B_S_FREE = 18,      // [2]
+    B_P_FULL = 20,      // [2]
+    B_PV_DONE = 22,     // [2]
+    B_Q_FULL = 24,
+    B_Q_FREE = 25,
+    B_O_FREE = 26,
+    B_FINAL = 27,
 };
 
-// Tile k occupies page slots (2k) mod 5 and (2k + 1) mod 5; page p of the ring
-// sequence completes phase (p / 5) & 1 of its slot's barriers.
-__device__ __forceinline__ int slot_of(uint32_t page_seq) { return (int)(page_seq % kSlots); }
-__device__ __forceinline__ uint32_t phase_of(uint32_t page_seq) { return (page_seq / kSlots) & 1; }
-
+// Page (= tile) k of the ring sequence uses slot k mod 5 and completes phase (k / 5) & 1
+// of that slot's barriers.
+__device__ __forceinline__ int slot_of(uint32_t k) { return (int)(k % kSlots); }
+__device__ __forceinline__ uint32_t phase_of(uint32_t k) { return (k / kSlots) & 1; }
 
 // byte offset of 16-byte chunk c (0..3) of row r in a 64-byte-swizzled block
 __device__ __forceinline__ uint32_t sw64(int r, int c) { return (uint32_t)(r * 64 + (((c ^ (r >> 1)) & 3) << 4)); }
@@ -154,10 +152,10 @@ __device__ __forceinline__ void split_e4m3x2(float w0, float w1, uint32_t& hi, u
     hi = (uint32_t)c;
     lo = (uint32_t)__nv_cvt_halfraw2_to_fp8x2(*reinterpret_cast<const __half2_raw*>(&r), __NV_SATFINITE, __NV_E4M3);
 }
-// 32 weights -> two e4m3 terms, four codes per word
-__device__ __forceinline__ void split32(const float (&w)[32], uint32_t (&chi)[8], uint32_t (&clo)[8]) {
+// 16 weights -> two e4m3 terms, four codes per word
+__device__ __forceinline__ void split16(const float (&w)[16], uint32_t (&chi)[4], uint32_t (&clo)[4]) {
 #pragma unroll
-    for (int j = 0; j < 32; j += 4) {
+    for (int j = 0; j < 16; j += 4) {
         uint32_t h01, l01, h23, l23;
         split_e4m3x2(w[j], w[j + 1], h01, l01);
         split_e4m3x2(w[j + 2], w[j + 3], h23, l23);
@@ -225,14 +223,13 @@ __global__ void __launch_bounds__(128) mla_fp8_qsplit_kernel(const __nv_bfloat16
 template <int HQ>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_fp8_kernel(const __grid_constant__ CUtensorMap tmC, DecodeArgs a) {
-    constexpr uint32_t IDESC_S128 = umma::idesc_f8(umma::kE4M3, umma::kE4M3, 0, 0, 128, 128);
-    constexpr uint32_t IDESC_S64 = umma::idesc_f8(umma::kE4M3, umma::kE4M3, 0, 0, 128, 64);
+    constexpr uint32_t IDESC_S = umma::idesc_f8(umma::kE4M3, umma::kE4M3, 0, 0, 128, kPg);
     constexpr uint32_t IDESC_PV = umma::idesc_f8(umma::kE4M3, umma::kE4M3, 1, 0, 128, HQ);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
     uint8_t* sm = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
     uint64_t* bar = reinterpret_cast<uint64_t*>(sm + kOffBars);
-    StageMeta* tmeta = reinterpret_cast<StageMeta*>(sm + kOffMeta);  // per page slot (a tile's first)
+    StageMeta* tmeta = reinterpret_cast<StageMeta*>(sm + kOffMeta);  // per page slot
     float* s_alpha = reinterpret_cast<float*>(sm + kOffSmall);
     float* s_inv = s_alpha + 64;
     float* s_gmax = s_inv + 64;     // [2 token groups][64 heads]
@@ -250,15 +247,15 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar + B_PAGE_EMPTY + i, 1);
         }
         for (int i = 0; i < 2; i++) {
+            mbar_init(bar + B_S_FULL + i, 1);
+            mbar_init(bar + B_S_FREE + i, kSoftWarps);
             mbar_init(bar + B_P_FULL + i, kSoftWarps);
             mbar_init(bar + B_PV_DONE + i, 1);
         }
-        mbar_init(bar + B_S_FULL, 1);
-        mbar_init(bar + B_S_FREE, kSoftWarps);
         mbar_init(bar + B_Q_FULL, kSoftWarps);
         mbar_init(bar + B_Q_FREE, 1);
         mbar_init(bar + B_O_FREE, kSoftWarps);
-        mbar_init(bar + B_FINAL, 1);
+        mbar_init(bar + B_FINAL, 2);
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -272,23 +269,22 @@ __global__ void __launch_bounds__(kThreads, 1)
     umma::fence_after_sync();
     const uint32_t tmem = *reinterpret_cast<volatile uint32_t*>(s_misc);
     const uint32_t t_o = tmem + kColO;  // O^T: columns [blk*HQ, blk*HQ + HQ)
-    const uint32_t t_s = tmem + kColS;  // S: 128 token columns
+    const uint32_t t_s = tmem + kColS;  // S buffers: [kColS + 64 sb, +64)
     const uint32_t t_q = tmem + kColQ;  // query rows, first 512 columns (128 TMEM columns)
     const int num_units = a.plan->num_units;
     const int P = a.page_size;
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
-        // Pages go into the slot ring one by one, each as soon as its slot is free.  One
-        // tile of lookahead: the next tile's unit and page indices are fetched before the
-        // waits, so their latency overlaps them.  Lane 0 takes tickets and handles the
-        // barriers; lanes 0..8 then issue a page's nine boxes and lane 9 its scales at once.
+        // One page of lookahead: the next page's unit and index are fetched before the slot
+        // wait, so their latency overlaps it.  Lane 0 takes tickets and handles the barriers;
+        // lanes 0..8 then issue the page's nine boxes and lane 9 its scales at once.
         const uint64_t pol = l2_policy_evict_first();
         if (lane == 0) tma_prefetch_desc(&tmC);
         int ui = -1, k = 0, nt = 0;
         Unit u;
         u.n = u.b = u.t0 = u.t1 = u.slot = u.n_chunks = u.slot_base = u.pad = 0;
-        // moves (ui, k) to the next tile (the same on every lane); false when no work is left
+        // moves (ui, k) to the next page (the same on every lane); false when no work is left
         auto advance = [&]() -> bool {
             if (ui >= 0 && k + 1 < nt) {
                 k++;
@@ -299,196 +295,138 @@ __global__ void __launch_bounds__(kThreads, 1)
             ui = __shfl_sync(0xffffffffu, nu, 0);
             if (ui >= num_units) return false;
             u = a.units[ui];
-            nt = max(1, (u.t1 - u.t0 + kT - 1) / kT);  // an empty unit still yields one tile
+            nt = max(1, (u.t1 - u.t0 + kPg - 1) / kPg);  // an empty unit still yields one tile
             k = 0;
             return true;
         };
-        auto pages = [&](int& p0, int& p1) {
-            const int t = u.t0 + k * kT;
-            const int nv = max(0, min(u.t1 - t, kT));
-            p0 = nv > 0 ? page_of(a, u.n, u.b, t / P) : -1;
-            p1 = nv > kPg ? page_of(a, u.n, u.b, t / P + 1) : -1;
+        auto page = [&]() -> int {
+            const int t = u.t0 + k * kPg;
+            return (u.t1 - t > 0) ? page_of(a, u.n, u.b, t / P) : -1;
         };
         bool have = advance();
-        int pg0 = -1, pg1 = -1;
-        if (have) pages(pg0, pg1);
+        int pg = have ? page() : -1;
         uint32_t ps = 0;  // pages issued into the ring
-        bool ok = true;
-        while (ok) {
+        while (true) {
             const bool c_have = have;
-            const int c_ui = ui, c_k = k, c_nt = nt, c_pg0 = pg0, c_pg1 = pg1;
+            const int c_ui = ui, c_k = k, c_nt = nt, c_pg = pg;
             const Unit c_u = u;
             if (have) {
                 have = advance();
-                if (have) pages(pg0, pg1);
+                if (have) pg = page();
             }
-            const int t = c_u.t0 + c_k * kT;
-            int nvalid = c_have ? max(0, min(c_u.t1 - t, kT)) : 0;
-            const int npages = (nvalid + kPg - 1) / kPg;
-            if ((npages > 0 && c_pg0 < 0) || (npages > 1 && c_pg1 < 0)) {
+            const int slot = slot_of(ps);
+            int waited = 1;
+            if (lane == 0) waited = mbar_wait(bar + B_PAGE_EMPTY + slot, phase_of(ps) ^ 1, s_abort, a.status);
+            if (!__shfl_sync(0xffffffffu, waited, 0)) break;
+            if (lane == 0) TRACE(14, ps);
+            if (!c_have) {
+                if (lane == 0) {
+                    tmeta[slot] = StageMeta{-1, 0, 0, 0};
+                    mbar_arrive(bar + B_PAGE_FULL + slot);
+                }
+                break;
+            }
+            const int t = c_u.t0 + c_k * kPg;
+            int nvalid = max(0, min(c_u.t1 - t, kPg));
+            if (nvalid > 0 && c_pg < 0) {
                 if (lane == 0) record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
                 nvalid = 0;
             }
             const int flags = (c_k == 0 ? kStageFirst : 0) | (c_k == c_nt - 1 ? kStageLast : 0);
-            for (int g = 0; g < 2; g++, ps++) {
-                const int slot = slot_of(ps);
-                int waited = 1;
-                if (lane == 0) waited = mbar_wait(bar + B_PAGE_EMPTY + slot, phase_of(ps) ^ 1, s_abort, a.status);
-                if (!__shfl_sync(0xffffffffu, waited, 0)) {
-                    ok = false;
-                    break;
-                }
-                if (lane == 0) TRACE(14, ps / 2);
-                if (g == 0) {
-                    if (lane == 0)
-                        tmeta[slot] = c_have ? StageMeta{c_ui, t, flags | (nvalid << 8), c_k} : StageMeta{-1, 0, 0, 0};
-                    if (!c_have) {
-                        if (lane == 0) mbar_arrive(bar + B_PAGE_FULL + slot);
-                        ok = false;
-                        break;
-                    }
-                }
-                if (nvalid > g * kPg) {
-                    if (lane == 0) mbar_arrive_expect_tx(bar + B_PAGE_FULL + slot, kPageBytes + kPg * 4);
-                    __syncwarp();
-                    const int32_t row0 = (g ? c_pg1 : c_pg0) * P;
-                    if (lane < kKB)
-                        tma_load_2d(sm + kOffTiles + slot * kBox + lane * kKbStride, &tmC, lane * 64, row0,
-                                    bar + B_PAGE_FULL + slot, pol);
-                    else if (lane == kKB)
-                        bulk_g2s(sm + kOffScales + slot * kPg * 4, a.kv_scales + row0, kPg * 4,
-                                 bar + B_PAGE_FULL + slot);
-                } else if (lane == 0) {
-                    mbar_arrive(bar + B_PAGE_FULL + slot);
-                }
-                if (lane == 0) TRACE(15, ps / 2);
+            if (lane == 0) tmeta[slot] = StageMeta{c_ui, t, flags | (nvalid << 8), c_k};
+            if (nvalid > 0) {
+                if (lane == 0) mbar_arrive_expect_tx(bar + B_PAGE_FULL + slot, kTileBytes + kPg * 4);
+                __syncwarp();
+                const int32_t row0 = c_pg * P;
+                if (lane < kKB)
+                    tma_load_2d(sm + kOffTiles + slot * kTileBytes + lane * kBox, &tmC, lane * 64, row0,
+                                bar + B_PAGE_FULL + slot, pol);
+                else if (lane == kKB)
+                    bulk_g2s(sm + kOffScales + slot * kPg * 4, a.kv_scales + row0, kPg * 4, bar + B_PAGE_FULL + slot);
+            } else if (lane == 0) {
+                mbar_arrive(bar + B_PAGE_FULL + slot);
             }
+            if (lane == 0) TRACE(15, ps);
+            ps++;
         }
         if (lane == 0 && *s_abort) {  // bounded drain of copies still in flight
             const uint32_t n = ps < (uint32_t)kSlots ? ps : (uint32_t)kSlots;
             for (uint32_t i = 1; i <= n; i++)
                 mbar_wait(bar + B_PAGE_FULL + slot_of(ps - i), phase_of(ps - i), nullptr, a.status);
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer (event loop)
+    } else if (warp == 1 || warp == 2 + kSoftWarps) {
+        // ------------------------------------------------------------------ MMA issuers
+        // Two threads: warp 1 issues the scores of each page as soon as its page, its S buffer
+        // and its unit's query rows are ready; the last warp issues P V of each page when the
+        // softmax has written its weights.  Each thread's waits hide behind the other's MMAs.
         if (lane == 0) {
-            const uint64_t dr0 = umma::smem_desc(sm_u32 + kOffRope, 16, 512, umma::kSw64);
-            const uint64_t dt0 = umma::smem_desc(sm_u32 + kOffTiles, 16, 512, umma::kSw64);
-            const uint64_t dv0 = umma::smem_desc(sm_u32 + kOffTiles, kKbStride, 512, umma::kSw64);
-            const uint64_t dp0 = umma::smem_desc(sm_u32 + kOffP, 16, 512, umma::kSw64);
-            uint32_t next_s = 0, next_pv = 0, unit_k = 0, ofree_k = 0;
-            uint32_t first_bits = 0;  // bit b: tile with parity b opened its unit
-            bool sentinel = false;
-            uint64_t t_prog = global_timer_ns();
-            while (true) {
-                bool progress = false;
-                if (next_pv < next_s) {
-                    const int pb = next_pv & 1;
-                    const bool fst = (first_bits >> pb) & 1;
-                    if (mbar_test(bar + B_P_FULL + pb, (next_pv >> 1) & 1) &&
-                        (!fst || mbar_test(bar + B_O_FREE, (ofree_k & 1) ^ 1))) {
-                        if (fst) ofree_k++;
-                        TRACE(2, next_pv);
-                        umma::fence_after_sync();
-                        // page by page, so that the first page's slot is released early; consecutive
-                        // MMAs go to different accumulator blocks
-#pragma unroll
-                        for (int g = 0; g < 2; g++) {
-                            const int sl = slot_of(2 * next_pv + g);
-#pragma unroll
-                            for (int j = 0; j < 2; j++)
-#pragma unroll
-                                for (int ks = 0; ks < 2; ks++)
-#pragma unroll
-                                    for (int blk = 0; blk < 4; blk++) {
-                                        const uint64_t ad =
-                                            dv0 + (uint64_t)((sl * kBox + 2 * blk * kKbStride + ks * 2048) >> 4);
-                                        const uint64_t bd =
-                                            dp0 + (uint64_t)((pb * kPBuf + j * kPTerm + g * 4096 + ks * 32) >> 4);
-                                        umma::mma_f8(t_o + blk * HQ, ad, bd, IDESC_PV,
-                                                     (fst && j == 0 && g == 0 && ks == 0) ? 0u : 1u);
-                                    }
-                            umma::commit(bar + B_PAGE_EMPTY + sl);
-                        }
-                        umma::commit(bar + B_PV_DONE + pb);
-                        TRACE(4, next_pv);
-                        next_pv++;
-                        progress = true;
-                    }
-                }
-                // S(k) needs its two pages, the S columns read out by the softmax (tile k-1)
-                // and the query rows of its unit
-                if (!sentinel && next_s - next_pv < 2 &&
-                    (next_s == 0 || mbar_test(bar + B_S_FREE, (next_s - 1) & 1))) {
-                    const uint32_t p0 = 2 * next_s, p1 = p0 + 1;
-                    const int s0 = slot_of(p0), s1 = slot_of(p1);
-                    if (mbar_test(bar + B_PAGE_FULL + s0, phase_of(p0))) {
-                        const StageMeta meta = load_meta(tmeta + s0);
-                        if (meta.unit < 0) {
-                            sentinel = true;
-                        } else if (mbar_test(bar + B_PAGE_FULL + s1, phase_of(p1))) {
-                            const bool first = meta.flags & kStageFirst;
-                            if (!first || mbar_test(bar + B_Q_FULL, unit_k & 1)) {
-                                if (first) unit_k++;
-                                TRACE(0, next_s);
-                                umma::fence_after_sync();
-                                if (s1 == s0 + 1) {
-                                    // adjacent slots: one 128-row operand
-                                    const uint32_t tile = (uint32_t)(s0 * kBox);
-#pragma unroll
-                                    for (int kb = 0; kb < 8; kb++)
-#pragma unroll
-                                        for (int ks = 0; ks < 2; ks++)
-                                            umma::mma_f8_ts(t_s, t_q + (2 * kb + ks) * 8,
-                                                            dt0 + (uint64_t)((tile + kb * kKbStride + ks * 32) >> 4),
-                                                            IDESC_S128, (kb | ks) ? 1u : 0u);
-#pragma unroll
-                                    for (int ks = 0; ks < 2; ks++)
-                                        umma::mma_f8(t_s, dr0 + (uint64_t)((ks * 32) >> 4),
-                                                     dt0 + (uint64_t)((tile + 8 * kKbStride + ks * 32) >> 4),
-                                                     IDESC_S128, 1u);
-                                } else {
-                                    // the ring wraps between the two pages: two 64-row halves
-#pragma unroll
-                                    for (int g = 0; g < 2; g++) {
-                                        const uint32_t tile = (uint32_t)((g ? s1 : s0) * kBox);
-#pragma unroll
-                                        for (int kb = 0; kb < 8; kb++)
-#pragma unroll
-                                            for (int ks = 0; ks < 2; ks++)
-                                                umma::mma_f8_ts(t_s + 64 * g, t_q + (2 * kb + ks) * 8,
-                                                                dt0 + (uint64_t)((tile + kb * kKbStride + ks * 32) >> 4),
-                                                                IDESC_S64, (kb | ks) ? 1u : 0u);
-#pragma unroll
-                                        for (int ks = 0; ks < 2; ks++)
-                                            umma::mma_f8(t_s + 64 * g, dr0 + (uint64_t)((ks * 32) >> 4),
-                                                         dt0 + (uint64_t)((tile + 8 * kKbStride + ks * 32) >> 4),
-                                                         IDESC_S64, 1u);
-                                    }
-                                }
-                                umma::commit(bar + B_S_FULL);
-                                if (meta.flags & kStageLast) umma::commit(bar + B_Q_FREE);
-                                TRACE(1, next_s);
-                                const int ts = next_s & 1;
-                                first_bits = (first_bits & ~(1u << ts)) | ((first ? 1u : 0u) << ts);
-                                next_s++;
-                                progress = true;
-                            }
-                        }
-                    }
-                }
-                if (sentinel && next_pv == next_s) break;
-                if (progress) {
-                    t_prog = global_timer_ns();
-                } else {
-                    // nothing ready: yield the issue slots this warp shares with softmax warps
-                    __nanosleep(32);
-                    if (*s_abort) break;
-                    if (global_timer_ns() - t_prog > kWaitLimitNs) {
-                        record_status(a.status, DCP_ERR_TIMEOUT);
-                        *s_abort = 1;
+            uint32_t unit_k = 0, ofree_k = 0;
+            if (warp == 1) {
+                const uint64_t dr0 = umma::smem_desc(sm_u32 + kOffRope, 16, 512, umma::kSw64);
+                const uint64_t dt0 = umma::smem_desc(sm_u32 + kOffTiles, 16, 512, umma::kSw64);
+                for (uint32_t kk = 0;; kk++) {
+                    const int slot = slot_of(kk);
+                    if (!mbar_wait(bar + B_PAGE_FULL + slot, phase_of(kk), s_abort, a.status)) break;
+                    const StageMeta meta = load_meta(tmeta + slot);
+                    if (meta.unit < 0) break;
+                    if (kk >= 2 &&
+                        !mbar_wait(bar + B_S_FREE + (kk & 1), ((kk - 2) >> 1) & 1, s_abort, a.status))
                         break;
+                    if (meta.flags & kStageFirst) {
+                        if (!mbar_wait(bar + B_Q_FULL, unit_k & 1, s_abort, a.status)) break;
+                        unit_k++;
                     }
+                    TRACE(0, kk);
+                    umma::fence_after_sync();
+                    const int sb = kk & 1;
+                    const uint64_t dt = dt0 + (uint64_t)((slot * kTileBytes) >> 4);
+#pragma unroll
+                    for (int kb = 0; kb < 8; kb++)
+#pragma unroll
+                        for (int ks = 0; ks < 2; ks++)
+                            umma::mma_f8_ts(t_s + sb * kPg, t_q + (2 * kb + ks) * 8,
+                                            dt + (uint64_t)((kb * kBox + ks * 32) >> 4), IDESC_S, (kb | ks) ? 1u : 0u);
+#pragma unroll
+                    for (int ks = 0; ks < 2; ks++)
+                        umma::mma_f8(t_s + sb * kPg, dr0 + (uint64_t)((ks * 32) >> 4),
+                                     dt + (uint64_t)((8 * kBox + ks * 32) >> 4), IDESC_S, 1u);
+                    umma::commit(bar + B_S_FULL + sb);
+                    if (meta.flags & kStageLast) umma::commit(bar + B_Q_FREE);
+                    TRACE(1, kk);
+                }
+            } else {
+                const uint64_t dv0 = umma::smem_desc(sm_u32 + kOffTiles, kBox, 512, umma::kSw64);
+                const uint64_t dp0 = umma::smem_desc(sm_u32 + kOffP, 16, 512, umma::kSw64);
+                for (uint32_t kk = 0;; kk++) {
+                    const int slot = slot_of(kk);
+                    // the page's metadata stays in place until this thread releases the slot
+                    if (!mbar_wait(bar + B_PAGE_FULL + slot, phase_of(kk), s_abort, a.status)) break;
+                    const StageMeta meta = load_meta(tmeta + slot);
+                    if (meta.unit < 0) break;
+                    const int pb = kk & 1;
+                    if (!mbar_wait(bar + B_P_FULL + pb, (kk >> 1) & 1, s_abort, a.status)) break;
+                    const bool fst = meta.flags & kStageFirst;
+                    if (fst) {
+                        if (!mbar_wait(bar + B_O_FREE, (ofree_k & 1) ^ 1, s_abort, a.status)) break;
+                        ofree_k++;
+                    }
+                    TRACE(2, kk);
+                    umma::fence_after_sync();
+                    const uint64_t da = dv0 + (uint64_t)((slot * kTileBytes) >> 4);
+                    const uint64_t db = dp0 + (uint64_t)((pb * kPBuf) >> 4);
+                    // consecutive MMAs go to different accumulator blocks
+#pragma unroll
+                    for (int j = 0; j < 2; j++)
+#pragma unroll
+                        for (int ks = 0; ks < 2; ks++)
+#pragma unroll
+                            for (int blk = 0; blk < 4; blk++)
+                                umma::mma_f8(t_o + blk * HQ, da + (uint64_t)((2 * blk * kBox + ks * 2048) >> 4),
+                                             db + (uint64_t)((j * kPTerm + ks * 32) >> 4), IDESC_PV,
+                                             (fst && j == 0 && ks == 0) ? 0u : 1u);
+                    umma::commit(bar + B_PAGE_EMPTY + slot);
+                    umma::commit(bar + B_PV_DONE + pb);
+                    TRACE(4, kk);
                 }
             }
             umma::commit(bar + B_FINAL);
@@ -497,12 +435,12 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------------ query rows, softmax, epilogue
         const int qd = warp & 3;                  // TMEM lane quadrant
-        const int wg = (warp - 2) >> 2;           // token group: tile tokens 64 wg .. 64 wg + 63 (page wg)
+        const int wg = (warp - 2) >> 2;           // token group: page tokens 32 wg .. 32 wg + 31
         const int half = lane >> 4;               // 0: row holds S_hi; 1: S_lo
         const int h = 16 * qd + (lane & 15);      // head
         const bool head = h < HQ;
         const int row = 32 * qd + lane;           // query row = TMEM lane
-        const int base = 64 * wg + 32 * half;     // my 32 tokens of the tile
+        const int base = 32 * wg + 16 * half;     // my 16 tokens of the page
         const int tid = threadIdx.x - 64;         // 0..255
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
         uint32_t seq = 0, unit_k = 0;
@@ -511,18 +449,17 @@ __global__ void __launch_bounds__(kThreads, 1)
         Unit u;
         u.n = u.b = u.t0 = u.t1 = u.slot = u.n_chunks = u.slot_base = u.pad = 0;
         while (true) {
-            const int ts = seq & 1;
-            const int s0 = slot_of(2 * seq), s1 = slot_of(2 * seq + 1);
-            if (!fail) fail = !mbar_wait(bar + B_PAGE_FULL + s0, phase_of(2 * seq), s_abort, a.status);
+            const int sb = seq & 1;
+            const int slot = slot_of(seq);
+            if (!fail) fail = !mbar_wait(bar + B_PAGE_FULL + slot, phase_of(seq), s_abort, a.status);
             StageMeta meta{-1, 0, 0, 0};
-            if (!fail) meta = load_meta(tmeta + s0);
+            if (!fail) meta = load_meta(tmeta + slot);
             if (named_barrier_or(kSmBar, 256, fail)) break;
             if (meta.unit < 0) break;
             const bool first = meta.flags & kStageFirst;
             const bool last = meta.flags & kStageLast;
             const int nvalid = (meta.flags >> 8) & 0xFF;
-            const bool full = nvalid == kT;
-            const int my_slot = wg ? s1 : s0;  // page holding my tokens
+            const bool full = nvalid == kPg;
             if (first) {
                 u = a.units[meta.unit];
                 f = head ? __ldg(a.qinv + (int64_t)u.b * 64 + h) * a.scale_log2 : 0.f;
@@ -567,29 +504,29 @@ __global__ void __launch_bounds__(kThreads, 1)
                 o_has = false;
             }
             // ---- scores: rows S_hi (lane < 16) and S_lo (lane >= 16) of head h; swap halves
-            if (!fail) fail = !mbar_wait(bar + B_S_FULL, seq & 1, s_abort, a.status);
+            if (!fail) fail = !mbar_wait(bar + B_S_FULL + sb, (seq >> 1) & 1, s_abort, a.status);
             umma::fence_after_sync();
             if (threadIdx.x == 64) TRACE(5, seq);
-            const float4* tsc4 = reinterpret_cast<const float4*>(sm + kOffScales + my_slot * kPg * 4 + 32 * half * 4);
-            float x[32];
+            if (lane == 0) TRACE(24 + warp - 2, seq);
+            const float4* tsc4 = reinterpret_cast<const float4*>(sm + kOffScales + (slot * kPg + base) * 4);
+            float x[16];
             float smax = 0.f;
             {
-                uint32_t v0[32], v1[32];
-                umma::ld32(t_s + lane_off + 64 * wg, v0);
-                umma::ld32(t_s + lane_off + 64 * wg + 32, v1);
+                uint32_t v[32];
+                umma::ld32(t_s + lane_off + sb * kPg + 32 * wg, v);
                 umma::wait_ld();
-                // the S columns may be overwritten by the next tile's MMAs from here on
+                // this S buffer may be overwritten by page seq+2 from here on
                 umma::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar + B_S_FREE);
+                if (lane == 0) mbar_arrive(bar + B_S_FREE + sb);
 #pragma unroll
-                for (int j4 = 0; j4 < 8; j4++) {
+                for (int j4 = 0; j4 < 4; j4++) {
                     const float4 sc4 = tsc4[j4];
                     const float sc[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
                         const int j = 4 * j4 + e;
-                        const uint32_t keep = half ? v1[j] : v0[j], send = half ? v0[j] : v1[j];
+                        const uint32_t keep = half ? v[16 + j] : v[j], send = half ? v[j] : v[16 + j];
                         const float s =
                             __uint_as_float(keep) + __uint_as_float(__shfl_xor_sync(0xffffffffu, send, 16));
                         x[j] = s * f * sc[e];
@@ -600,7 +537,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     // tokens past the end of the unit: no score, and their stale scales do not count
                     smax = 0.f;
 #pragma unroll
-                    for (int j4 = 0; j4 < 8; j4++) {
+                    for (int j4 = 0; j4 < 4; j4++) {
                         const float4 sc4 = tsc4[j4];
                         const float sc[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
 #pragma unroll
@@ -615,7 +552,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (threadIdx.x == 64) TRACE(6, seq);
             float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 32; j++) mx = fmaxf(mx, x[j]);
+            for (int j = 0; j < 16; j++) mx = fmaxf(mx, x[j]);
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
             // combine with the other token group of the same heads
@@ -642,9 +579,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (any && *s_abort) break;
             if (threadIdx.x == 64) TRACE(8, seq);
             if (any) {
-                // the previous tile's P V must be complete before O^T is rescaled; token group wg
+                // the previous page's P V must be complete before O^T is rescaled; token group wg
                 // rescales value blocks 2 wg, 2 wg + 1 of its lane quadrant
-                fail = !mbar_wait(bar + B_PV_DONE + (ts ^ 1), ((seq - 1) >> 1) & 1, s_abort, a.status);
+                fail = !mbar_wait(bar + B_PV_DONE + (sb ^ 1), ((seq - 1) >> 1) & 1, s_abort, a.status);
                 if (!fail) {
                     umma::fence_after_sync();
 #pragma unroll 1
@@ -663,16 +600,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma::wait_st();
                 }
             }
-            // ---- W = p s_t as two e4m3 terms (the P buffer is free once P V of tile seq-2 is done)
-            if (!fail) fail = !mbar_wait(bar + B_PV_DONE + ts, ((seq >> 1) & 1) ^ 1, s_abort, a.status);
+            // ---- W = p s_t as two e4m3 terms (the P buffer is free once P V of page seq-2 is done)
+            if (!fail) fail = !mbar_wait(bar + B_PV_DONE + sb, ((seq >> 1) & 1) ^ 1, s_abort, a.status);
             if (threadIdx.x == 64) TRACE(10, seq);
             if (!fail && head) {
-                float w[32];
+                float w[16];
                 float rowsum = 0.f;
                 if (m_used != -INFINITY) {
                     // 2^(-inf - m) = 0 for masked tokens; stale scales are zeroed below
 #pragma unroll
-                    for (int j4 = 0; j4 < 8; j4++) {
+                    for (int j4 = 0; j4 < 4; j4++) {
                         const float4 sc4 = tsc4[j4];
                         const float sc[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
 #pragma unroll
@@ -684,49 +621,45 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (!full) {
 #pragma unroll
-                        for (int j = 0; j < 32; j++) w[j] = (base + j < nvalid) ? w[j] : 0.f;
+                        for (int j = 0; j < 16; j++) w[j] = (base + j < nvalid) ? w[j] : 0.f;
                     }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 32; j++) w[j] = 0.f;
+                    for (int j = 0; j < 16; j++) w[j] = 0.f;
                 }
-                uint32_t chi[8], clo[8];
-                split32(w, chi, clo);
+                uint32_t chi[4], clo[4];
+                split16(w, chi, clo);
                 lpart = lpart * alpha + rowsum;
-                // page wg of the tile, row h, 16-byte chunks 2 half and 2 half + 1
-                uint8_t* pb = sm + kOffP + ts * kPBuf + wg * 4096;
-#pragma unroll
-                for (int cc = 0; cc < 2; cc++) {
-                    const int c = 2 * half + cc;
-                    *reinterpret_cast<uint4*>(pb + sw64(h, c)) =
-                        make_uint4(chi[4 * cc], chi[4 * cc + 1], chi[4 * cc + 2], chi[4 * cc + 3]);
-                    *reinterpret_cast<uint4*>(pb + kPTerm + sw64(h, c)) =
-                        make_uint4(clo[4 * cc], clo[4 * cc + 1], clo[4 * cc + 2], clo[4 * cc + 3]);
-                }
+                // row h, 16-byte chunk 2 wg + half = my tokens
+                uint8_t* pb = sm + kOffP + sb * kPBuf;
+                const uint32_t off = sw64(h, 2 * wg + half);
+                *reinterpret_cast<uint4*>(pb + off) = make_uint4(chi[0], chi[1], chi[2], chi[3]);
+                *reinterpret_cast<uint4*>(pb + kPTerm + off) = make_uint4(clo[0], clo[1], clo[2], clo[3]);
             } else if (!fail) {
                 lpart = lpart * alpha;
             }
             if (!fail && !full) {
                 // rows past the last valid token hold stale page bytes (possibly NaN codes):
                 // zero their value columns so that W = 0 cannot meet them
-                const int nr = kT - nvalid;
+                uint8_t* tile = sm + kOffTiles + slot * kTileBytes;
+                const int nr = kPg - nvalid;
                 for (int i = tid; i < nr * 4 * 8; i += 256) {
                     const int kb = i / (nr * 4), rem = i - kb * nr * 4;
-                    const int tok = nvalid + rem / 4, c = rem & 3;
-                    *reinterpret_cast<uint4*>(sm + kOffTiles + kb * kKbStride + (tok < kPg ? s0 : s1) * kBox +
-                                              (tok % kPg) * 64 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+                    const int r = nvalid + rem / 4, c = rem & 3;
+                    *reinterpret_cast<uint4*>(tile + kb * kBox + r * 64 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
             umma::fence_proxy_async_smem();
             umma::fence_before_sync();
             __syncwarp();
-            if (!fail && lane == 0) mbar_arrive(bar + B_P_FULL + ts);
+            if (!fail && lane == 0) mbar_arrive(bar + B_P_FULL + sb);
             if (threadIdx.x == 64) TRACE(9, seq);
+            if (lane == 0) TRACE(16 + warp - 2, seq);
             o_has = true;
             // ---- end of unit: O = O^T / l, LSE
             if (last) {
                 if (threadIdx.x == 64) TRACE(12, seq);
-                if (!fail) fail = !mbar_wait(bar + B_PV_DONE + ts, (seq >> 1) & 1, s_abort, a.status);
+                if (!fail) fail = !mbar_wait(bar + B_PV_DONE + sb, (seq >> 1) & 1, s_abort, a.status);
                 umma::fence_after_sync();
                 const float lg = lpart + __shfl_xor_sync(0xffffffffu, lpart, 16);  // this token group
                 if (half == 0) s_gl[wg * 64 + h] = lg;
