@@ -18,34 +18,36 @@
 // in one warp's TMEM lane quadrant.  The first 512 columns of those rows live
 // in tensor memory (the MMA's A operand), the 64 rope columns in shared memory.
 //
-// Scores.  [S_hi; S_lo] = [Q_hi; Q_lo] . C^T per page, M = 128, N = 64 tokens,
-// K = 576: 16 MMAs with A in TMEM + 2 with A in shared memory; the page is the
-// only shared-memory operand.  Lane pairs (l, l + 16) swap halves with shuffles
-// and form s = scale * s_t * (S_hi + S_lo) / sigma_h.
+// Scores.  [S_hi; S_lo] = [Q_hi; Q_lo] . C^T, M = 128, K = 576, over a tile of
+// one or two pages (N = 64 or 128 tokens): 16 MMAs with A in TMEM + 2 with A in
+// shared memory; the pages are the only shared-memory operand.  Lane pairs
+// (l, l + 16) swap halves with shuffles and form
+// s = scale * s_t * (S_hi + S_lo) / sigma_h.
 //
-// Values.  O^T = V^T . W^T with V^T read MN-major straight from the raw page
+// Values.  O^T = V^T . W^T with V^T read MN-major straight from the raw pages
 // and W = p * s_t in two e4m3 terms (relative error below 2^-8).  The running
-// maximum m absorbs the page's largest scale (m >= max_t (x_t + log2 s_t), x in
+// maximum m absorbs the tile's largest scale (m >= max_t (x_t + log2 s_t), x in
 // log2 units), so W = 2^(x - m) s_t <= 2^8 stays inside e4m3's range whatever
 // the scales; it is rescaled lazily (O^T only when m grows by more than 2^8).
-//   O^T += V^T . W_j^T   M = 128 value columns (4 blocks), N = Hq, K = 64, j = 0, 1
+//   O^T += V^T . W_j^T   M = 128 value columns (4 blocks), N = Hq, K = 64 per page, j = 0, 1
 // 16 MMAs per page.  O = O^T / l with l = sum_t 2^(x_t - m).
 //
-// Pages: nine [64 rows][64 B] TMA boxes with 64-byte swizzle (36 KB) + 256 B
-// of scales, in a ring of five slots; a slot is refilled as soon as P V of its
-// page completes.
+// Pages: nine [64 rows][64 B] TMA boxes with 64-byte swizzle (36 KB) + 256 B of
+// scales, in a ring of five slots laid out [block][slot][64 rows][64 B], so that
+// two adjacent slots form one 128-row operand.  A tile pairs a page with the next
+// one unless the page sits in the last slot or closes its unit.  A slot is
+// refilled as soon as P V of its page completes.
 //
 // Warp roles (one CTA per SM, persistent, units from an atomic ticket):
 //   warp 0      producer: tickets, page indices (one page of lookahead), TMA
-//   warp 1      TMEM allocation; issues the scores of each page
+//   warp 1      TMEM allocation; issues the scores of each tile
 //   warps 2..9  query rows, softmax, lazy rescale of O^T, epilogue.  The two
 //               warps on TMEM quadrant j own heads 16 j .. 16 j + 15: warp
-//               group g (warps 2..5: g = 0, 6..9: g = 1) the page's tokens
-//               32 g .. 32 g + 31, in which lane l < 16 takes the first 16
-//               and lane l + 16 the last 16; g also picks the value blocks
-//               2 g, 2 g + 1 that the warp rescales and stores.
-//   warp 10     issues P V of each page
-// Scores run up to two pages ahead of the softmax (two S buffers in TMEM).
+//               group g (warps 2..5: g = 0, 6..9: g = 1) page g of the tile,
+//               in which lane l < 16 takes tokens 0..31 and lane l + 16 tokens
+//               32..63; g also picks the value blocks 2 g, 2 g + 1 that the warp
+//               rescales and stores.
+//   warp 10     issues P V of each tile
 #include "common.cuh"
 #include "finish.cuh"
 #include "kernels.h"
@@ -78,9 +80,11 @@ constexpr int kKB = 9;                     // 576 = 9 blocks of 64 bytes
 constexpr int kBox = kPg * 64;             // [64 rows][64 B] box: 4 KB
 constexpr int kTileBytes = kKB * kBox;     // one page: 36864
 constexpr int kSlots = 5;                  // pages in flight
+constexpr int kKbStride = kSlots * kBox;   // block kb of every slot is contiguous: [kb][slot][64 rows][64 B]
 constexpr int kRopeBytes = 128 * 64;       // rope columns of the 128 query rows
-constexpr int kPTerm = 64 * 64;            // W_j^T [64 heads][64 tokens] e4m3: 4 KB
-constexpr int kPBuf = 2 * kPTerm;          // 8 KB
+constexpr int kPTerm = 64 * 64;            // W_j^T of one page [64 heads][64 tokens] e4m3: 4 KB
+constexpr int kPPage = 2 * kPTerm;         // both terms of one page
+constexpr int kPBuf = 2 * kPPage;          // a tile of two pages: 16 KB
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kSmBar = 1;                  // the 256 softmax threads
 constexpr int kPairBar = 2;                // + quadrant: the two warps sharing a TMEM lane quadrant
@@ -103,8 +107,8 @@ static_assert(kOffRope % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands need
 enum : int {
     B_PAGE_FULL = 0,    // [kSlots]
     B_PAGE_EMPTY = 8,   // [kSlots]
-    B_S_FULL = 16,      // [2]
-    B_S_FREE = 18,      // [2]
+    B_S_FULL = 16,
+    B_S_FREE = 17,
     B_P_FULL = 20,      // [2]
     B_PV_DONE = 22,     // [2]
     B_Q_FULL = 24,
@@ -152,16 +156,23 @@ __device__ __forceinline__ void split_e4m3x2(float w0, float w1, uint32_t& hi, u
     hi = (uint32_t)c;
     lo = (uint32_t)__nv_cvt_halfraw2_to_fp8x2(*reinterpret_cast<const __half2_raw*>(&r), __NV_SATFINITE, __NV_E4M3);
 }
-// 16 weights -> two e4m3 terms, four codes per word
-__device__ __forceinline__ void split16(const float (&w)[16], uint32_t (&chi)[4], uint32_t (&clo)[4]) {
+// 32 weights -> two e4m3 terms, four codes per word
+__device__ __forceinline__ void split32(const float (&w)[32], uint32_t (&chi)[8], uint32_t (&clo)[8]) {
 #pragma unroll
-    for (int j = 0; j < 16; j += 4) {
+    for (int j = 0; j < 32; j += 4) {
         uint32_t h01, l01, h23, l23;
         split_e4m3x2(w[j], w[j + 1], h01, l01);
         split_e4m3x2(w[j + 2], w[j + 3], h23, l23);
         chi[j / 4] = h01 | (h23 << 16);
         clo[j / 4] = l01 | (l23 << 16);
     }
+}
+
+// A tile is one page, or two when the page is not in the last slot (so the next page's
+// slot is adjacent) and does not close its unit.  Producer order makes the next page the
+// next one of the same unit then.
+__device__ __forceinline__ bool pairs_with_next(int slot, const StageMeta& m) {
+    return slot != kSlots - 1 && !(m.flags & kStageLast);
 }
 
 // ------------------------------------------------------------------------------------------
@@ -224,6 +235,7 @@ template <int HQ>
 __global__ void __launch_bounds__(kThreads, 1)
     mla_fp8_kernel(const __grid_constant__ CUtensorMap tmC, DecodeArgs a) {
     constexpr uint32_t IDESC_S = umma::idesc_f8(umma::kE4M3, umma::kE4M3, 0, 0, 128, kPg);
+    constexpr uint32_t IDESC_S128 = umma::idesc_f8(umma::kE4M3, umma::kE4M3, 0, 0, 128, 2 * kPg);
     constexpr uint32_t IDESC_PV = umma::idesc_f8(umma::kE4M3, umma::kE4M3, 1, 0, 128, HQ);
 
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -247,11 +259,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             mbar_init(bar + B_PAGE_EMPTY + i, 1);
         }
         for (int i = 0; i < 2; i++) {
-            mbar_init(bar + B_S_FULL + i, 1);
-            mbar_init(bar + B_S_FREE + i, kSoftWarps);
             mbar_init(bar + B_P_FULL + i, kSoftWarps);
             mbar_init(bar + B_PV_DONE + i, 1);
         }
+        mbar_init(bar + B_S_FULL, 1);
+        mbar_init(bar + B_S_FREE, kSoftWarps);
         mbar_init(bar + B_Q_FULL, kSoftWarps);
         mbar_init(bar + B_Q_FREE, 1);
         mbar_init(bar + B_O_FREE, kSoftWarps);
@@ -339,7 +351,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 const int32_t row0 = c_pg * P;
                 if (lane < kKB)
-                    tma_load_2d(sm + kOffTiles + slot * kTileBytes + lane * kBox, &tmC, lane * 64, row0,
+                    tma_load_2d(sm + kOffTiles + lane * kKbStride + slot * kBox, &tmC, lane * 64, row0,
                                 bar + B_PAGE_FULL + slot, pol);
                 else if (lane == kKB)
                     bulk_g2s(sm + kOffScales + slot * kPg * 4, a.kv_scales + row0, kPg * 4, bar + B_PAGE_FULL + slot);
@@ -364,69 +376,81 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (warp == 1) {
                 const uint64_t dr0 = umma::smem_desc(sm_u32 + kOffRope, 16, 512, umma::kSw64);
                 const uint64_t dt0 = umma::smem_desc(sm_u32 + kOffTiles, 16, 512, umma::kSw64);
-                for (uint32_t kk = 0;; kk++) {
+                for (uint32_t kk = 0, tt = 0;; tt++) {
                     const int slot = slot_of(kk);
                     if (!mbar_wait(bar + B_PAGE_FULL + slot, phase_of(kk), s_abort, a.status)) break;
-                    const StageMeta meta = load_meta(tmeta + slot);
-                    if (meta.unit < 0) break;
-                    if (kk >= 2 &&
-                        !mbar_wait(bar + B_S_FREE + (kk & 1), ((kk - 2) >> 1) & 1, s_abort, a.status))
-                        break;
-                    if (meta.flags & kStageFirst) {
+                    const StageMeta m0 = load_meta(tmeta + slot);
+                    if (m0.unit < 0) break;
+                    const bool pair = pairs_with_next(slot, m0);
+                    StageMeta m1 = m0;
+                    if (pair) {
+                        if (!mbar_wait(bar + B_PAGE_FULL + slot + 1, phase_of(kk + 1), s_abort, a.status)) break;
+                        m1 = load_meta(tmeta + slot + 1);
+                    }
+                    // the softmax has read the previous tile's scores
+                    if (tt >= 1 && !mbar_wait(bar + B_S_FREE, (tt - 1) & 1, s_abort, a.status)) break;
+                    if (m0.flags & kStageFirst) {
                         if (!mbar_wait(bar + B_Q_FULL, unit_k & 1, s_abort, a.status)) break;
                         unit_k++;
                     }
-                    TRACE(0, kk);
+                    TRACE(0, tt);
                     umma::fence_after_sync();
-                    const int sb = kk & 1;
-                    const uint64_t dt = dt0 + (uint64_t)((slot * kTileBytes) >> 4);
+                    const uint32_t idesc = pair ? IDESC_S128 : IDESC_S;
+                    const uint64_t dt = dt0 + (uint64_t)((slot * kBox) >> 4);
 #pragma unroll
                     for (int kb = 0; kb < 8; kb++)
 #pragma unroll
                         for (int ks = 0; ks < 2; ks++)
-                            umma::mma_f8_ts(t_s + sb * kPg, t_q + (2 * kb + ks) * 8,
-                                            dt + (uint64_t)((kb * kBox + ks * 32) >> 4), IDESC_S, (kb | ks) ? 1u : 0u);
+                            umma::mma_f8_ts(t_s, t_q + (2 * kb + ks) * 8, dt + (uint64_t)((kb * kKbStride + ks * 32) >> 4),
+                                            idesc, (kb | ks) ? 1u : 0u);
 #pragma unroll
                     for (int ks = 0; ks < 2; ks++)
-                        umma::mma_f8(t_s + sb * kPg, dr0 + (uint64_t)((ks * 32) >> 4),
-                                     dt + (uint64_t)((8 * kBox + ks * 32) >> 4), IDESC_S, 1u);
-                    umma::commit(bar + B_S_FULL + sb);
-                    if (meta.flags & kStageLast) umma::commit(bar + B_Q_FREE);
-                    TRACE(1, kk);
+                        umma::mma_f8(t_s, dr0 + (uint64_t)((ks * 32) >> 4),
+                                     dt + (uint64_t)((8 * kKbStride + ks * 32) >> 4), idesc, 1u);
+                    umma::commit(bar + B_S_FULL);
+                    if (m1.flags & kStageLast) umma::commit(bar + B_Q_FREE);
+                    TRACE(1, tt);
+                    kk += pair ? 2 : 1;
                 }
             } else {
-                const uint64_t dv0 = umma::smem_desc(sm_u32 + kOffTiles, kBox, 512, umma::kSw64);
+                const uint64_t dv0 = umma::smem_desc(sm_u32 + kOffTiles, kKbStride, 512, umma::kSw64);
                 const uint64_t dp0 = umma::smem_desc(sm_u32 + kOffP, 16, 512, umma::kSw64);
-                for (uint32_t kk = 0;; kk++) {
+                for (uint32_t kk = 0, tt = 0;; tt++) {
                     const int slot = slot_of(kk);
                     // the page's metadata stays in place until this thread releases the slot
                     if (!mbar_wait(bar + B_PAGE_FULL + slot, phase_of(kk), s_abort, a.status)) break;
-                    const StageMeta meta = load_meta(tmeta + slot);
-                    if (meta.unit < 0) break;
-                    const int pb = kk & 1;
-                    if (!mbar_wait(bar + B_P_FULL + pb, (kk >> 1) & 1, s_abort, a.status)) break;
-                    const bool fst = meta.flags & kStageFirst;
+                    const StageMeta m0 = load_meta(tmeta + slot);
+                    if (m0.unit < 0) break;
+                    const bool pair = pairs_with_next(slot, m0);
+                    const int pb = tt & 1;
+                    if (!mbar_wait(bar + B_P_FULL + pb, (tt >> 1) & 1, s_abort, a.status)) break;
+                    const bool fst = m0.flags & kStageFirst;
                     if (fst) {
                         if (!mbar_wait(bar + B_O_FREE, (ofree_k & 1) ^ 1, s_abort, a.status)) break;
                         ofree_k++;
                     }
-                    TRACE(2, kk);
+                    TRACE(2, tt);
                     umma::fence_after_sync();
-                    const uint64_t da = dv0 + (uint64_t)((slot * kTileBytes) >> 4);
-                    const uint64_t db = dp0 + (uint64_t)((pb * kPBuf) >> 4);
-                    // consecutive MMAs go to different accumulator blocks
+                    for (int g = 0; g < (pair ? 2 : 1); g++) {
+                        const int sl = slot + g;
+                        const uint64_t da = dv0 + (uint64_t)((sl * kBox) >> 4);
+                        const uint64_t db = dp0 + (uint64_t)((pb * kPBuf + g * kPPage) >> 4);
+                        // consecutive MMAs go to different accumulator blocks
 #pragma unroll
-                    for (int j = 0; j < 2; j++)
+                        for (int j = 0; j < 2; j++)
 #pragma unroll
-                        for (int ks = 0; ks < 2; ks++)
+                            for (int ks = 0; ks < 2; ks++)
 #pragma unroll
-                            for (int blk = 0; blk < 4; blk++)
-                                umma::mma_f8(t_o + blk * HQ, da + (uint64_t)((2 * blk * kBox + ks * 2048) >> 4),
-                                             db + (uint64_t)((j * kPTerm + ks * 32) >> 4), IDESC_PV,
-                                             (fst && j == 0 && ks == 0) ? 0u : 1u);
-                    umma::commit(bar + B_PAGE_EMPTY + slot);
+                                for (int blk = 0; blk < 4; blk++)
+                                    umma::mma_f8(t_o + blk * HQ,
+                                                 da + (uint64_t)((2 * blk * kKbStride + ks * 2048) >> 4),
+                                                 db + (uint64_t)((j * kPTerm + ks * 32) >> 4), IDESC_PV,
+                                                 (fst && g == 0 && j == 0 && ks == 0) ? 0u : 1u);
+                        umma::commit(bar + B_PAGE_EMPTY + sl);
+                    }
                     umma::commit(bar + B_PV_DONE + pb);
-                    TRACE(4, kk);
+                    TRACE(4, tt);
+                    kk += pair ? 2 : 1;
                 }
             }
             umma::commit(bar + B_FINAL);
@@ -435,36 +459,45 @@ __global__ void __launch_bounds__(kThreads, 1)
     } else {
         // ------------------------------------------------------------------ query rows, softmax, epilogue
         const int qd = warp & 3;                  // TMEM lane quadrant
-        const int wg = (warp - 2) >> 2;           // token group: page tokens 32 wg .. 32 wg + 31
+        const int wg = (warp - 2) >> 2;           // token group = page wg of the tile
         const int half = lane >> 4;               // 0: row holds S_hi; 1: S_lo
         const int h = 16 * qd + (lane & 15);      // head
         const bool head = h < HQ;
         const int row = 32 * qd + lane;           // query row = TMEM lane
-        const int base = 32 * wg + 16 * half;     // my 16 tokens of the page
+        const int base = 32 * half;               // my 32 tokens of the page
         const int tid = threadIdx.x - 64;         // 0..255
+        const int gtid = tid & 127;               // index within the token group
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
-        uint32_t seq = 0, unit_k = 0;
+        uint32_t seq = 0, kk = 0, unit_k = 0;
         float m_used = -INFINITY, lpart = 0.f, f = 0.f;
         bool o_has = false, fail = false;
         Unit u;
         u.n = u.b = u.t0 = u.t1 = u.slot = u.n_chunks = u.slot_base = u.pad = 0;
         while (true) {
-            const int sb = seq & 1;
-            const int slot = slot_of(seq);
-            if (!fail) fail = !mbar_wait(bar + B_PAGE_FULL + slot, phase_of(seq), s_abort, a.status);
-            StageMeta meta{-1, 0, 0, 0};
-            if (!fail) meta = load_meta(tmeta + slot);
+            const int pb = seq & 1;
+            const int slot0 = slot_of(kk);
+            if (!fail) fail = !mbar_wait(bar + B_PAGE_FULL + slot0, phase_of(kk), s_abort, a.status);
+            StageMeta m0{-1, 0, 0, 0};
+            if (!fail) m0 = load_meta(tmeta + slot0);
             if (named_barrier_or(kSmBar, 256, fail)) break;
-            if (meta.unit < 0) break;
-            const bool first = meta.flags & kStageFirst;
-            const bool last = meta.flags & kStageLast;
-            const int nvalid = (meta.flags >> 8) & 0xFF;
+            if (m0.unit < 0) break;
+            const bool pair = pairs_with_next(slot0, m0);
+            StageMeta m1 = m0;
+            if (pair) {
+                if (!fail) fail = !mbar_wait(bar + B_PAGE_FULL + slot0 + 1, phase_of(kk + 1), s_abort, a.status);
+                if (!fail) m1 = load_meta(tmeta + slot0 + 1);
+            }
+            const bool first = m0.flags & kStageFirst;
+            const bool last = m1.flags & kStageLast;
+            const bool mine = wg == 0 || pair;          // does my page exist in this tile
+            const int my_slot = mine ? slot0 + wg : slot0;
+            const int nvalid = mine ? (((wg ? m1.flags : m0.flags) >> 8) & 0xFF) : 0;
             const bool full = nvalid == kPg;
             if (first) {
-                u = a.units[meta.unit];
+                u = a.units[m0.unit];
                 f = head ? __ldg(a.qinv + (int64_t)u.b * 64 + h) * a.scale_log2 : 0.f;
                 // the previous unit's S MMAs are complete (first unit passes at once)
-                fail = !mbar_wait(bar + B_Q_FREE, (unit_k & 1) ^ 1, s_abort, a.status);
+                fail = fail || !mbar_wait(bar + B_Q_FREE, (unit_k & 1) ^ 1, s_abort, a.status);
                 if (!fail) {
                     if (head) {
                         // token group wg copies query bytes [256 wg, 256 wg + 256) -> TMEM columns 64 wg ..
@@ -503,41 +536,43 @@ __global__ void __launch_bounds__(kThreads, 1)
                 lpart = 0.f;
                 o_has = false;
             }
-            // ---- scores: rows S_hi (lane < 16) and S_lo (lane >= 16) of head h; swap halves
-            if (!fail) fail = !mbar_wait(bar + B_S_FULL + sb, (seq >> 1) & 1, s_abort, a.status);
+            // ---- scores of my page: rows S_hi (lane < 16) and S_lo (lane >= 16) of head h; swap halves
+            if (!fail) fail = !mbar_wait(bar + B_S_FULL, seq & 1, s_abort, a.status);
             umma::fence_after_sync();
             if (threadIdx.x == 64) TRACE(5, seq);
             if (lane == 0) TRACE(24 + warp - 2, seq);
-            const float4* tsc4 = reinterpret_cast<const float4*>(sm + kOffScales + (slot * kPg + base) * 4);
-            float x[16];
+            const float4* tsc4 = reinterpret_cast<const float4*>(sm + kOffScales + (my_slot * kPg + base) * 4);
+            float x[32];
             float smax = 0.f;
             {
-                uint32_t v[32];
-                umma::ld32(t_s + lane_off + sb * kPg + 32 * wg, v);
+                uint32_t v0[32], v1[32];
+                umma::ld32(t_s + lane_off + 64 * wg, v0);
+                umma::ld32(t_s + lane_off + 64 * wg + 32, v1);
                 umma::wait_ld();
-                // this S buffer may be overwritten by page seq+2 from here on
+                // the S columns may be overwritten by the next tile's MMAs from here on
                 umma::fence_before_sync();
                 __syncwarp();
-                if (lane == 0) mbar_arrive(bar + B_S_FREE + sb);
+                if (lane == 0) mbar_arrive(bar + B_S_FREE);
 #pragma unroll
-                for (int j4 = 0; j4 < 4; j4++) {
+                for (int j4 = 0; j4 < 8; j4++) {
                     const float4 sc4 = tsc4[j4];
                     const float sc[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
                         const int j = 4 * j4 + e;
-                        const uint32_t keep = half ? v[16 + j] : v[j], send = half ? v[j] : v[16 + j];
-                        const float s =
+                        const uint32_t keep = half ? v1[j] : v0[j], send = half ? v0[j] : v1[j];
+                        const float sv =
                             __uint_as_float(keep) + __uint_as_float(__shfl_xor_sync(0xffffffffu, send, 16));
-                        x[j] = s * f * sc[e];
+                        x[j] = sv * f * sc[e];
                         smax = fmaxf(smax, sc[e]);
                     }
                 }
                 if (!full) {
-                    // tokens past the end of the unit: no score, and their stale scales do not count
+                    // tokens past the end of the unit (or no page): no score, and their stale
+                    // scales do not count
                     smax = 0.f;
 #pragma unroll
-                    for (int j4 = 0; j4 < 4; j4++) {
+                    for (int j4 = 0; j4 < 8; j4++) {
                         const float4 sc4 = tsc4[j4];
                         const float sc[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
 #pragma unroll
@@ -552,10 +587,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (threadIdx.x == 64) TRACE(6, seq);
             float mx = -INFINITY;
 #pragma unroll
-            for (int j = 0; j < 16; j++) mx = fmaxf(mx, x[j]);
+            for (int j = 0; j < 32; j++) mx = fmaxf(mx, x[j]);
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
-            // combine with the other token group of the same heads
+            // combine with the other page of the tile (same heads)
             if (half == 0) {
                 s_gmax[wg * 64 + h] = mx;
                 s_gsmax[wg * 64 + h] = smax;
@@ -579,9 +614,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (any && *s_abort) break;
             if (threadIdx.x == 64) TRACE(8, seq);
             if (any) {
-                // the previous page's P V must be complete before O^T is rescaled; token group wg
+                // the previous tile's P V must be complete before O^T is rescaled; token group wg
                 // rescales value blocks 2 wg, 2 wg + 1 of its lane quadrant
-                fail = !mbar_wait(bar + B_PV_DONE + (sb ^ 1), ((seq - 1) >> 1) & 1, s_abort, a.status);
+                fail = !mbar_wait(bar + B_PV_DONE + (pb ^ 1), ((seq - 1) >> 1) & 1, s_abort, a.status);
                 if (!fail) {
                     umma::fence_after_sync();
 #pragma unroll 1
@@ -600,16 +635,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                     umma::wait_st();
                 }
             }
-            // ---- W = p s_t as two e4m3 terms (the P buffer is free once P V of page seq-2 is done)
-            if (!fail) fail = !mbar_wait(bar + B_PV_DONE + sb, ((seq >> 1) & 1) ^ 1, s_abort, a.status);
+            // ---- W = p s_t as two e4m3 terms (the P buffer is free once P V of tile seq-2 is done)
+            if (!fail) fail = !mbar_wait(bar + B_PV_DONE + pb, ((seq >> 1) & 1) ^ 1, s_abort, a.status);
             if (threadIdx.x == 64) TRACE(10, seq);
-            if (!fail && head) {
-                float w[16];
+            if (!fail && head && mine) {
+                float w[32];
                 float rowsum = 0.f;
                 if (m_used != -INFINITY) {
                     // 2^(-inf - m) = 0 for masked tokens; stale scales are zeroed below
 #pragma unroll
-                    for (int j4 = 0; j4 < 4; j4++) {
+                    for (int j4 = 0; j4 < 8; j4++) {
                         const float4 sc4 = tsc4[j4];
                         const float sc[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
 #pragma unroll
@@ -621,45 +656,51 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (!full) {
 #pragma unroll
-                        for (int j = 0; j < 16; j++) w[j] = (base + j < nvalid) ? w[j] : 0.f;
+                        for (int j = 0; j < 32; j++) w[j] = (base + j < nvalid) ? w[j] : 0.f;
                     }
                 } else {
 #pragma unroll
-                    for (int j = 0; j < 16; j++) w[j] = 0.f;
+                    for (int j = 0; j < 32; j++) w[j] = 0.f;
                 }
-                uint32_t chi[4], clo[4];
-                split16(w, chi, clo);
+                uint32_t chi[8], clo[8];
+                split32(w, chi, clo);
                 lpart = lpart * alpha + rowsum;
-                // row h, 16-byte chunk 2 wg + half = my tokens
-                uint8_t* pb = sm + kOffP + sb * kPBuf;
-                const uint32_t off = sw64(h, 2 * wg + half);
-                *reinterpret_cast<uint4*>(pb + off) = make_uint4(chi[0], chi[1], chi[2], chi[3]);
-                *reinterpret_cast<uint4*>(pb + kPTerm + off) = make_uint4(clo[0], clo[1], clo[2], clo[3]);
+                // page wg of the tile, row h, 16-byte chunks 2 half and 2 half + 1
+                uint8_t* pbuf = sm + kOffP + pb * kPBuf + wg * kPPage;
+#pragma unroll
+                for (int cc = 0; cc < 2; cc++) {
+                    const uint32_t off = sw64(h, 2 * half + cc);
+                    *reinterpret_cast<uint4*>(pbuf + off) =
+                        make_uint4(chi[4 * cc], chi[4 * cc + 1], chi[4 * cc + 2], chi[4 * cc + 3]);
+                    *reinterpret_cast<uint4*>(pbuf + kPTerm + off) =
+                        make_uint4(clo[4 * cc], clo[4 * cc + 1], clo[4 * cc + 2], clo[4 * cc + 3]);
+                }
             } else if (!fail) {
                 lpart = lpart * alpha;
             }
-            if (!fail && !full) {
+            if (!fail && mine && !full) {
                 // rows past the last valid token hold stale page bytes (possibly NaN codes):
-                // zero their value columns so that W = 0 cannot meet them
-                uint8_t* tile = sm + kOffTiles + slot * kTileBytes;
+                // zero their value columns so that W = 0 cannot meet them (token group wg
+                // clears its own page)
+                uint8_t* tile = sm + kOffTiles + my_slot * kBox;
                 const int nr = kPg - nvalid;
-                for (int i = tid; i < nr * 4 * 8; i += 256) {
+                for (int i = gtid; i < nr * 4 * 8; i += 128) {
                     const int kb = i / (nr * 4), rem = i - kb * nr * 4;
                     const int r = nvalid + rem / 4, c = rem & 3;
-                    *reinterpret_cast<uint4*>(tile + kb * kBox + r * 64 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
+                    *reinterpret_cast<uint4*>(tile + kb * kKbStride + r * 64 + c * 16) = make_uint4(0u, 0u, 0u, 0u);
                 }
             }
             umma::fence_proxy_async_smem();
             umma::fence_before_sync();
             __syncwarp();
-            if (!fail && lane == 0) mbar_arrive(bar + B_P_FULL + sb);
+            if (!fail && lane == 0) mbar_arrive(bar + B_P_FULL + pb);
             if (threadIdx.x == 64) TRACE(9, seq);
             if (lane == 0) TRACE(16 + warp - 2, seq);
             o_has = true;
             // ---- end of unit: O = O^T / l, LSE
             if (last) {
                 if (threadIdx.x == 64) TRACE(12, seq);
-                if (!fail) fail = !mbar_wait(bar + B_PV_DONE + sb, (seq >> 1) & 1, s_abort, a.status);
+                if (!fail) fail = !mbar_wait(bar + B_PV_DONE + pb, (seq >> 1) & 1, s_abort, a.status);
                 umma::fence_after_sync();
                 const float lg = lpart + __shfl_xor_sync(0xffffffffu, lpart, 16);  // this token group
                 if (half == 0) s_gl[wg * 64 + h] = lg;
@@ -709,6 +750,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             if (threadIdx.x == 64) TRACE(11, seq);
             seq++;
+            kk += pair ? 2 : 1;
         }
     }
 
