@@ -24,6 +24,8 @@ collective.  Timing is the max over ranks of the device time.
 from __future__ import annotations
 
 import argparse
+import datetime
+import hashlib
 import json
 import os
 import statistics
@@ -47,7 +49,7 @@ HEADLINE_CONFIG = 5
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--steps", type=int, default=50)
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=HEADLINE_CONFIG)
@@ -90,7 +92,10 @@ def workload_config(w, args):
 # ----------------------------------------------------------------------------
 
 class Clocks:
-    Q = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+    """nvidia-smi sampling every 10 ms, started before the warm-up so that it is
+    running when the timed region begins; only samples whose timestamp falls
+    inside the timed region (host wall clock around it) are kept."""
+    Q = ("timestamp,index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
          "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
          "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
 
@@ -98,18 +103,23 @@ class Clocks:
         self.gpu = gpu_index
         self.f = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
         self.p = None
+        self.window = None
 
     def start(self):
         try:
             self.p = subprocess.Popen(["nvidia-smi", "-i", str(self.gpu), f"--query-gpu={self.Q}",
-                                       "--format=csv,noheader,nounits", "-lms", "200"], stdout=self.f,
+                                       "--format=csv,noheader,nounits", "-lms", "10"], stdout=self.f,
                                       stderr=subprocess.DEVNULL)
         except (OSError, FileNotFoundError):
             self.p = None
 
+    def mark(self, t0: float, t1: float):
+        """Host wall-clock bounds of the timed region."""
+        self.window = (t0, t1)
+
     def stop(self):
         if self.p is None:
-            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+            return {"sm_mhz": None, "sm_max_mhz": None, "samples": 0, "reasons": ["nvidia-smi unavailable"]}
         self.p.terminate()
         try:
             self.p.wait(timeout=5)
@@ -118,22 +128,82 @@ class Clocks:
         self.f.flush()
         rows = [r.split(",") for r in open(self.f.name).read().strip().splitlines() if r.strip()]
         os.unlink(self.f.name)
-        sm, mx, reasons = [], None, set()
-        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
-        for r in rows:
-            r = [x.strip() for x in r]
-            if len(r) < 9:
-                continue
-            try:
-                sm.append(float(r[1]))
-                mx = float(r[2])
-            except ValueError:
-                continue
-            for nm, v in zip(names, r[5:9]):
-                if v.lower() == "active":
-                    reasons.add(nm)
-        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "samples": len(sm),
-                "reasons": sorted(reasons)}
+        return summarize_clocks(rows, self.window)
+
+
+def summarize_clocks(rows, window):
+    """rows: nvidia-smi CSV fields (timestamp first); window: (t0, t1) epoch seconds or None."""
+    sm, mx, reasons = [], None, set()
+    names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+    for r in rows:
+        r = [x.strip() for x in r]
+        if len(r) < 10:
+            continue
+        try:
+            ts = datetime.datetime.strptime(r[0], "%Y/%m/%d %H:%M:%S.%f").timestamp()
+            clk, cmax = float(r[2]), float(r[3])
+        except ValueError:
+            continue
+        if window is not None and not (window[0] <= ts <= window[1]):
+            continue
+        sm.append(clk)
+        mx = cmax
+        for nm, v in zip(names, r[6:10]):
+            if v.lower() == "active":
+                reasons.add(nm)
+    return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": mx, "samples": len(sm),
+            "reasons": sorted(reasons)}
+
+
+# ----------------------------------------------------------------------------
+# DRAM traffic of the decode launch, from an ncu capture (profiles/)
+# ----------------------------------------------------------------------------
+
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_dram_traffic.json")
+KERNEL_SOURCES = os.path.join(ROOT, "sequence_sharded_paged_b200", "csrc")
+
+
+def kernel_sources_digest() -> str:
+    """sha256 over the CUDA sources of the library (a changed kernel voids old counters)."""
+    h = hashlib.sha256()
+    for name in sorted(os.listdir(KERNEL_SOURCES)):
+        if name.endswith((".cu", ".cuh", ".h")):
+            h.update(name.encode())
+            h.update(open(os.path.join(KERNEL_SOURCES, name), "rb").read())
+    return h.hexdigest()
+
+
+def measured_traffic(config_key: str):
+    """dram bytes read + written per decode launch, or None when no capture of
+    the current sources exists for this workload."""
+    if not os.path.exists(TRAFFIC_FILE):
+        return None
+    d = json.load(open(TRAFFIC_FILE))
+    if d.get("sources_sha256") != kernel_sources_digest():
+        return None
+    e = d.get("workloads", {}).get(config_key)
+    return None if e is None else float(e["dram_bytes_per_launch"])
+
+
+def traffic_key(args, w) -> str:
+    return f"config{args.config} B{w.B} N{w.n_shards} I{w.interleave}"
+
+
+def launches_per_step(w) -> int:
+    """Kernels one step launches: shard map, append, plan, [query split], decode, merge."""
+    fp8_tc = w.kind == "mla" and w.dtype == "fp8" and w.hq in (16, 32, 64) and w.page_size == 64
+    return 6 if fp8_tc else 5
+
+
+def combine_ranks(dist, device, ms, kern_total, e2e_ms, bytes_timed, e2e_bytes):
+    """Max over ranks of the device times, sum over ranks of the bytes."""
+    import torch
+    t = torch.tensor([ms, kern_total, e2e_ms], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    tb = torch.tensor([float(bytes_timed), float(e2e_bytes)], dtype=torch.float64, device=device)
+    dist.all_reduce(tb, op=dist.ReduceOp.SUM)
+    (ms, kern_total, e2e_ms), (b, eb) = t.tolist(), tb.tolist()
+    return ms, kern_total, e2e_ms, b, eb
 
 
 # ----------------------------------------------------------------------------
@@ -192,6 +262,8 @@ def run_ours(args, rank, world, local_rank):
             ev[1].record(stream)
         dcp.dcp_merge(o_part, lse, out, lse_out)
 
+    clocks = Clocks(local_rank)
+    clocks.start()
     for s in range(args.warmup):
         step(s)
     torch.cuda.synchronize()
@@ -204,18 +276,19 @@ def run_ours(args, rank, world, local_rank):
     ev_k = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(args.steps)]
     t_start = torch.cuda.Event(enable_timing=True)
     t_stop = torch.cuda.Event(enable_timing=True)
-    clocks = Clocks(local_rank)
     if world > 1:
         dist.barrier()
     torch.cuda.synchronize()
-    clocks.start()
+    wall0 = time.time()
     t_start.record(stream)
     for i in range(args.steps):
         step(args.warmup + i, ev_k[i])
     t_stop.record(stream)
     torch.cuda.synchronize()
+    wall1 = time.time()
     if world > 1:
         dist.barrier()
+    clocks.mark(wall0, wall1)
     clk = clocks.stop()
     st = dcp.dcp_get_device_status()
     if st != dcp.DCP_OK:
@@ -269,12 +342,8 @@ def run_ours(args, rank, world, local_rank):
 
     # max over ranks of device time; whole-job bytes
     if world > 1:
-        t = torch.tensor([ms, sum(kern_ms), e2e[0] if e2e else 0.0], device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        ms, kern_total, e2e_ms_max = t.tolist()
-        tb = torch.tensor([float(bytes_timed), float(e2e[1] if e2e else 0)], device=dev, dtype=torch.float64)
-        dist.all_reduce(tb, op=dist.ReduceOp.SUM)
-        bytes_all, e2e_bytes_all = tb.tolist()
+        ms, kern_total, e2e_ms_max, bytes_all, e2e_bytes_all = combine_ranks(
+            dist, dev, ms, sum(kern_ms), e2e[0] if e2e else 0.0, bytes_timed, e2e[1] if e2e else 0)
     else:
         kern_total = sum(kern_ms)
         bytes_all = float(bytes_timed)
@@ -282,6 +351,7 @@ def run_ours(args, rank, world, local_rank):
         e2e_bytes_all = float(e2e[1]) if e2e else 0.0
 
     hbm, peak_kind = peaks()
+    traffic = measured_traffic(traffic_key(args, w))
     gbs = bytes_all / (ms * 1e-3) / 1e9
     # dominant kernel: the decode (plan + split-KV attention) of one step, CUDA events on its stream
     per_launch_bytes = bytes_timed / args.steps
@@ -305,12 +375,13 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded counter-based generator; lengths shaped like the agentic trace)",
         "config": workload_config(w, args) | {"parallelism": f"replicas x{world} (one independent batch per GPU)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
-                     "frac": round(achieved / hbm, 3), "traffic": None,
+                     "frac": round(achieved / hbm, 3), "traffic": traffic,
+                     "algorithmic_bytes_per_launch": int(per_launch_bytes),
                      "kernel": "dcp_decode_partial (planner + split-KV attention)",
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback 6650 GB/s"},
         "clocks": clk,
-        "gpu_launches": 5 * args.steps,
+        "gpu_launches": launches_per_step(w) * args.steps,
         "fill_seconds": round(fill_s, 2),
     }
     if e2e:
