@@ -230,6 +230,8 @@ bool decode_geometry(int kind, int dtype, int hq, int hkv, int dk, int dv, int p
     return false;
 }
 
+bool mla_umma_supported(int hq, int page_size) { return (hq == 16 || hq == 32 || hq == 64) && page_size == 64; }
+
 cudaError_t launch_decode(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s) {
     switch (g.path) {
         case DecodePath::GqaSimt:

@@ -297,6 +297,8 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (progress) {
                     t_prog = global_timer_ns();
                 } else {
+                    // nothing ready: yield the issue slots this warp shares with a softmax warp
+                    __nanosleep(32);
                     if (*s_abort) break;
                     if (global_timer_ns() - t_prog > kWaitLimitNs) {
                         record_status(a.status, DCP_ERR_TIMEOUT);
@@ -454,10 +456,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (last) {
                 if (!fail) fail = !mbar_wait(bar + B_PV_DONE + ts, par, s_abort, a.status);
                 umma::fence_after_sync();
-                if (head) {
-                    s_m[h] = m_used;
-                    s_l[h] = lsum;
-                }
+                if (head) s_l[h] = lsum > 0.f ? 1.f / lsum : 0.f;  // O = O^T * (1 / l)
                 if (named_barrier_or(kSmBar, 128, fail)) break;
                 const int64_t shard = (int64_t)u.n * a.batch + u.b;
                 const bool split = u.n_chunks > 1;
@@ -472,16 +471,11 @@ __global__ void __launch_bounds__(kThreads, 1)
                         umma::ld16(t_o + lane_off + blk * HQ + c0, r);
                         umma::wait_ld();
 #pragma unroll
-                        for (int i = 0; i < 16; i++) {
-                            const float l = s_l[c0 + i];
-                            __stcg(obase + (int64_t)(c0 + i) * 512 + dv, l > 0.f ? __uint_as_float(r[i]) / l : 0.f);
-                        }
+                        for (int i = 0; i < 16; i++)
+                            __stcg(obase + (int64_t)(c0 + i) * 512 + dv, __uint_as_float(r[i]) * s_l[c0 + i]);
                     }
                 }
-                if (head) {
-                    const float l = s_l[h];
-                    __stcg(lbase + h, l > 0.f ? (s_m[h] + log2f(l)) * kLn2 : -INFINITY);
-                }
+                if (head) __stcg(lbase + h, lsum > 0.f ? (m_used + log2f(lsum)) * kLn2 : -INFINITY);
                 umma::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar + B_O_FREE);

@@ -57,9 +57,8 @@ int simt_blocks_per_sm(DecodePath p, int D, int G, int P, bool fp8);
 bool gqa_mma_supported(int hq, int hkv, int dk);
 int gqa_mma_blocks_per_sm(int hq, int hkv, int dk);
 cudaError_t launch_decode_gqa_mma(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s);
+// shapes the tensor-core MLA kernels take (both dtypes): Hq in {16, 32, 64}, 64-token pages
 bool mla_umma_supported(int hq, int page_size);
-size_t mla_umma_smem_bytes(bool fp8);
-cudaError_t launch_decode_mla_umma(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_mla_bf16(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_mla_fp8(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s);
 
