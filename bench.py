@@ -59,7 +59,7 @@ def parse():
                     help="keep only the first B requests of the workload (small profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
-    ap.add_argument("--cpu-seconds", type=float, default=15.0, help="target CPU work of the oracle sample")
+    ap.add_argument("--cpu-seconds", type=float, default=25.0, help="target CPU work of the oracle sample")
     return ap.parse_args()
 
 
@@ -395,94 +395,64 @@ def run_ours(args, rank, world, local_rank):
 # the oracle on host cores (CPU baseline / reference arm)
 # ----------------------------------------------------------------------------
 
-def oracle_sample(w, cpu_seconds: float, rate_tok_s: float | None = None):
-    """Pick requests (shortest-first from a seeded shuffle) until the sample
-    holds about cpu_seconds of oracle work; returns (req_list, tokens)."""
-    # calibrated oracle throughput (tokens*heads per second per core, float64 two-pass)
+def _oracle_run(w, q64, reqs):
+    """The oracle as it stands: unsharded float64 decode attention of the listed
+    requests, reading the inputs from the counter-based generator in C."""
     import oracle
-    cores = oracle.num_threads()
-    per_tok = (w.hq * (w.dk + w.dv) * 2) if w.kind == "mla" else (w.hq * (w.dk + w.dv) * 2)
-    flops_s = 1.0e9 * cores if rate_tok_s is None else rate_tok_s
-    budget_tok = max(1000, int(cpu_seconds * flops_s / per_tok))
-    order = np.argsort(synth.bits(synth.key(w.seed_len, 7), np.arange(w.B)))
+    oracle.decode_synth(w.kind, w.dtype, w.seed_val, q64, w.lengths, w.scale, w.hkv, w.dk, w.dv,
+                        req_list=np.asarray(reqs, dtype=np.int64))
+
+
+def oracle_sample(w, cpu_seconds: float, q64):
+    """Requests (a seeded shuffle) holding about cpu_seconds of oracle work: the
+    shortest request is timed first and the rate extrapolated (conservatively:
+    more requests run more parallel work items)."""
+    order = [int(b) for b in np.argsort(synth.bits(synth.key(w.seed_len, 7), np.arange(w.B)))]
+    probe = min(order, key=lambda b: int(w.lengths[b]))
+    t0 = time.perf_counter()
+    _oracle_run(w, q64, [probe])
+    rate = max(1.0, int(w.lengths[probe])) / max(time.perf_counter() - t0, 1e-4)  # tokens per second
+    budget_tok = max(int(w.lengths[probe]), int(cpu_seconds * rate))
     reqs, tot = [], 0
     for b in order:
         if tot + int(w.lengths[b]) > budget_tok and reqs:
             continue
-        reqs.append(int(b))
+        reqs.append(b)
         tot += int(w.lengths[b])
         if tot >= budget_tok:
             break
     return sorted(reqs), tot
 
 
-def oracle_arrays(w, reqs):
-    """Dense float64 inputs of the sampled requests (generated untimed)."""
-    import oracle
-    Lmax = int(max(w.lengths[b] for b in reqs))
-    B = len(reqs)
-    q = synth.bf16_bits_to_f64(synth.q_bf16(w.seed_val, w.B, w.hq, w.dk))[reqs]
-    lens = np.array([w.lengths[b] for b in reqs], np.int64)
-    if w.kind == "gqa":
-        K = np.zeros((B, Lmax, w.hkv, w.dk))
-        V = np.zeros((B, Lmax, w.hkv, w.dv))
-        for i, b in enumerate(reqs):
-            K[i, :lens[i]] = synth.bf16_bits_to_f64(synth.kv_rows_bf16(w.seed_val, synth.T_K, b, np.arange(lens[i]),
-                                                                        w.hkv, w.dk))
-            V[i, :lens[i]] = synth.bf16_bits_to_f64(synth.kv_rows_bf16(w.seed_val, synth.T_V, b, np.arange(lens[i]),
-                                                                        w.hkv, w.dv))
-        return q, K, V, lens
-    K = np.zeros((B, Lmax, 576))
-    for i, b in enumerate(reqs):
-        rows = synth.kv_rows_bf16(w.seed_val, synth.T_LATENT, b, np.arange(lens[i]), 1, 576)[:, 0]
-        if w.dtype == "fp8":
-            codes, sc = oracle.quantize_rows_e4m3(rows)
-            K[i, :lens[i]] = _E4M3[codes] * sc.astype(np.float64)[:, None]
-        else:
-            K[i, :lens[i]] = synth.bf16_bits_to_f64(rows)
-    return q, K, None, lens
-
-
-_E4M3 = None
-
-
-def _init_e4m3():
-    global _E4M3
-    import oracle
-    _E4M3 = oracle.e4m3_table()
-
-
 def time_oracle(w, cpu_seconds: float):
     """Time the oracle (as it stands) on a bounded sample; returns dict."""
     import oracle
-    _init_e4m3()
-    reqs, tot = oracle_sample(w, cpu_seconds)
-    q, K, V, lens = oracle_arrays(w, reqs)
+    q64 = synth.bf16_bits_to_f64(synth.q_bf16(w.seed_val, w.B, w.hq, w.dk))
+    reqs, tot = oracle_sample(w, cpu_seconds, q64)
     t0 = time.perf_counter()
-    oracle.decode_arrays(w.kind, q, K, V, lens, w.scale, dv=w.dv)
+    _oracle_run(w, q64, reqs)
     dt = time.perf_counter() - t0
-    kv_bytes = int(lens.sum()) * w.kv_bytes_per_token
+    kv_bytes = tot * w.kv_bytes_per_token
     return {"value": round(kv_bytes / dt / 1e9, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
-            "sample": f"{len(reqs)} of {w.B} requests ({int(lens.sum())} tokens, all {w.hq} heads, unsharded "
-                      f"float64 decode attention), {dt:.1f} s"}, dt, kv_bytes
+            "sample": f"{len(reqs)} of {w.B} requests ({tot} tokens, all {w.hq} heads, unsharded "
+                      f"float64 decode attention, inputs read from the generator), {dt:.1f} s"}, dt, kv_bytes
 
 
 def run_reference(args):
     w = get_workload(args)
     per_step = max(1.0, min(20.0, 120.0 / max(1, args.steps + args.warmup)))
     import oracle
-    _init_e4m3()
-    reqs, tot = oracle_sample(w, per_step)
-    q, K, V, lens = oracle_arrays(w, reqs)
-    kv_bytes = int(lens.sum()) * w.kv_bytes_per_token
+    q64 = synth.bf16_bits_to_f64(synth.q_bf16(w.seed_val, w.B, w.hq, w.dk))
+    reqs, tot = oracle_sample(w, per_step, q64)
+    kv_bytes = tot * w.kv_bytes_per_token
     for _ in range(args.warmup):
-        oracle.decode_arrays(w.kind, q, K, V, lens, w.scale, dv=w.dv)
+        _oracle_run(w, q64, reqs)
     t0 = time.perf_counter()
     for _ in range(args.steps):
-        oracle.decode_arrays(w.kind, q, K, V, lens, w.scale, dv=w.dv)
+        _oracle_run(w, q64, reqs)
     dt = time.perf_counter() - t0
     gbs = kv_bytes * args.steps / dt / 1e9
-    sample = (f"each step: {len(reqs)} of {w.B} requests ({int(lens.sum())} tokens, all {w.hq} heads) "
+    sample = (f"each step: {len(reqs)} of {w.B} requests ({tot} tokens, all {w.hq} heads) "
               f"of the workload, unsharded float64 decode attention on host cores")
     return {
         "impl": "reference",
