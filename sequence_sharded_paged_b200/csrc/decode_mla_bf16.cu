@@ -64,7 +64,7 @@ constexpr int kQBytes = kKB * 64 * 128;   // Q padded to 64 rows: 73728
 constexpr int kStages = 2;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kSmBar = 1;                 // named barrier of the softmax warps
-constexpr int kThreads = 192;
+constexpr int kThreads = 224;              // producer, S issuer, softmax x 4, P V issuer
 constexpr int kPBytes = 64 * 128;         // P_lo^T [64 heads][64 tokens] bf16
 
 constexpr uint32_t kOffQ = 0;
@@ -134,7 +134,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar + B_Q_FULL, 4);
         mbar_init(bar + B_Q_FREE, 1);
         mbar_init(bar + B_O_FREE, 4);
-        mbar_init(bar + B_FINAL, 1);
+        mbar_init(bar + B_FINAL, 2);
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -219,92 +219,76 @@ __global__ void __launch_bounds__(kThreads, 1)
                 }
             }
         }
-    } else if (warp == 1) {
-        // ------------------------------------------------------------------ MMA issuer
+    } else if (warp == 1 || warp == 6) {
+        // ------------------------------------------------------------------ MMA issuers
+        // Two threads.  Warp 1 issues S of each tile once it has landed, the softmax has read
+        // the S buffer's previous tile (its P is ready) and (first tile of a unit) Q is loaded.
+        // Warp 6 issues P V of each tile once its P is ready; its completion frees the tile for
+        // the next load.  Each thread's waits hide behind the other's MMAs.
         if (lane == 0) {
-            const uint64_t dq0 = umma::smem_desc(sm_u32 + kOffQ, 16, 1024, umma::kSw128);
             const uint64_t dt0 = umma::smem_desc(sm_u32 + kOffTiles, 16, 1024, umma::kSw128);
-            const uint64_t dv0 = umma::smem_desc(sm_u32 + kOffTiles, kBox, 1024, umma::kSw128);
-            // Event loop: P V of the oldest tile is issued as soon as its P is ready (its
-            // completion frees the tile for the next load); S of the next tile as soon as it
-            // has landed, its S buffer is free and (first tile of a unit) Q is loaded.
-            uint32_t next_s = 0, next_pv = 0, unit_k = 0, ofree_k = 0;
-            uint32_t first_bits = 0;  // bit b: the tile in S buffer b opened its unit
-            bool sentinel = false;
-            uint64_t t_prog = global_timer_ns();
-            while (true) {
-                bool progress = false;
-                if (next_pv < next_s) {
-                    const int sb = next_pv & 1;
-                    if (mbar_test(bar + B_P_FULL + sb, (next_pv >> 1) & 1) &&
-                        (!((first_bits >> sb) & 1) || mbar_test(bar + B_O_FREE, (ofree_k & 1) ^ 1))) {
-                        TRACE(2, next_pv);
-                        const bool fst = (first_bits >> sb) & 1;
-                        if (fst) ofree_k++;
-                        umma::fence_after_sync();
-                        const uint64_t tile = (uint64_t)((sb * kTileBytes) >> 4);
-                        // P_hi^T sits in the tile's rope box, P_lo^T in its own buffer
-                        const uint64_t phi = dt0 + tile + (uint64_t)((8 * kBox) >> 4);
-                        const uint64_t plo = dt0 + (uint64_t)((kOffPlo - kOffTiles) >> 4);
-#pragma unroll
-                        for (int blk = 0; blk < 4; blk++)
-#pragma unroll
-                            for (int ks = 0; ks < kT / 16; ks++) {
-                                const uint64_t ad = dv0 + tile + (uint64_t)(((2 * blk) * kBox + ks * 2048) >> 4);
-                                umma::mma_f16(t_o + blk * HQ, ad, phi + (uint64_t)(ks * 2), IDESC_PV,
-                                              (fst && ks == 0) ? 0u : 1u);
-                                umma::mma_f16(t_o + blk * HQ, ad, plo + (uint64_t)(ks * 2), IDESC_PV, 1u);
-                            }
-                        umma::commit(bar + B_PV_DONE + sb);
-                        umma::commit(bar + B_TILE_EMPTY + sb);
-                        TRACE(4, next_pv);
-                        next_pv++;
-                        progress = true;
+            uint32_t unit_k = 0, ofree_k = 0;
+            if (warp == 1) {
+                const uint64_t dq0 = umma::smem_desc(sm_u32 + kOffQ, 16, 1024, umma::kSw128);
+                for (uint32_t k = 0;; k++) {
+                    const int ts = k & 1;
+                    if (!mbar_wait(bar + B_TILE_FULL + ts, (k >> 1) & 1, s_abort, a.status)) break;
+                    const StageMeta meta = load_meta(tmeta + ts);
+                    if (meta.unit < 0) break;
+                    if (k >= 2 && !mbar_wait(bar + B_P_FULL + ts, ((k - 2) >> 1) & 1, s_abort, a.status)) break;
+                    const bool first = meta.flags & kStageFirst;
+                    if (first) {
+                        if (!mbar_wait(bar + B_Q_FULL, unit_k & 1, s_abort, a.status)) break;
+                        unit_k++;
                     }
-                }
-                if (!sentinel && next_s - next_pv < 2) {
-                    const int ts = next_s & 1;
-                    if (mbar_test(bar + B_TILE_FULL + ts, (next_s >> 1) & 1)) {
-                        const StageMeta meta = load_meta(tmeta + ts);
-                        if (meta.unit < 0) {
-                            sentinel = true;
-                        } else {
-                            const bool first = meta.flags & kStageFirst;
-                            if (!first || mbar_test(bar + B_Q_FULL, unit_k & 1)) {
-                                TRACE(0, next_s);
-                                if (first) unit_k++;
-                                umma::fence_after_sync();
-                                const uint64_t tile = (uint64_t)((ts * kTileBytes) >> 4);
+                    TRACE(0, k);
+                    umma::fence_after_sync();
+                    const uint64_t tile = (uint64_t)((ts * kTileBytes) >> 4);
 #pragma unroll
-                                for (int kb = 0; kb < kKB; kb++)
+                    for (int kb = 0; kb < kKB; kb++)
 #pragma unroll
-                                    for (int ks = 0; ks < 4; ks++) {
-                                        const uint64_t off = (uint64_t)((kb * kBox + ks * 32) >> 4);
-                                        umma::mma_f16(t_s + ts * kT, dq0 + off, dt0 + tile + off, IDESC_S,
-                                                      (kb | ks) ? 1u : 0u);
-                                    }
-                                umma::commit(bar + B_S_FULL + ts);
-                                if (meta.flags & kStageLast) umma::commit(bar + B_Q_FREE);
-                                TRACE(1, next_s);
-                                first_bits = (first_bits & ~(1u << ts)) | ((first ? 1u : 0u) << ts);
-                                next_s++;
-                                progress = true;
-                            }
+                        for (int ks = 0; ks < 4; ks++) {
+                            const uint64_t off = (uint64_t)((kb * kBox + ks * 32) >> 4);
+                            umma::mma_f16(t_s + ts * kT, dq0 + off, dt0 + tile + off, IDESC_S, (kb | ks) ? 1u : 0u);
                         }
-                    }
+                    umma::commit(bar + B_S_FULL + ts);
+                    if (meta.flags & kStageLast) umma::commit(bar + B_Q_FREE);
+                    TRACE(1, k);
                 }
-                if (sentinel && next_pv == next_s) break;
-                if (progress) {
-                    t_prog = global_timer_ns();
-                } else {
-                    // nothing ready: yield the issue slots this warp shares with a softmax warp
-                    __nanosleep(32);
-                    if (*s_abort) break;
-                    if (global_timer_ns() - t_prog > kWaitLimitNs) {
-                        record_status(a.status, DCP_ERR_TIMEOUT);
-                        *s_abort = 1;
-                        break;
+            } else {
+                const uint64_t dv0 = umma::smem_desc(sm_u32 + kOffTiles, kBox, 1024, umma::kSw128);
+                for (uint32_t k = 0;; k++) {
+                    const int sb = k & 1;
+                    // the tile's metadata stays in place until this thread frees the tile
+                    if (!mbar_wait(bar + B_TILE_FULL + sb, (k >> 1) & 1, s_abort, a.status)) break;
+                    const StageMeta meta = load_meta(tmeta + sb);
+                    if (meta.unit < 0) break;
+                    if (!mbar_wait(bar + B_P_FULL + sb, (k >> 1) & 1, s_abort, a.status)) break;
+                    const bool fst = meta.flags & kStageFirst;
+                    if (fst) {
+                        if (!mbar_wait(bar + B_O_FREE, (ofree_k & 1) ^ 1, s_abort, a.status)) break;
+                        ofree_k++;
                     }
+                    TRACE(2, k);
+                    umma::fence_after_sync();
+                    const uint64_t tile = (uint64_t)((sb * kTileBytes) >> 4);
+                    // P_hi^T sits in the tile's rope box, P_lo^T in its own buffer; consecutive
+                    // MMAs go to different accumulator blocks
+                    const uint64_t phi = dt0 + tile + (uint64_t)((8 * kBox) >> 4);
+                    const uint64_t plo = dt0 + (uint64_t)((kOffPlo - kOffTiles) >> 4);
+#pragma unroll
+                    for (int ks = 0; ks < kT / 16; ks++)
+#pragma unroll
+                        for (int term = 0; term < 2; term++)
+#pragma unroll
+                            for (int blk = 0; blk < 4; blk++) {
+                                const uint64_t ad = dv0 + tile + (uint64_t)(((2 * blk) * kBox + ks * 2048) >> 4);
+                                umma::mma_f16(t_o + blk * HQ, ad, (term ? plo : phi) + (uint64_t)(ks * 2), IDESC_PV,
+                                              (fst && ks == 0 && term == 0) ? 0u : 1u);
+                            }
+                    umma::commit(bar + B_PV_DONE + sb);
+                    umma::commit(bar + B_TILE_EMPTY + sb);
+                    TRACE(4, k);
                 }
             }
             umma::commit(bar + B_FINAL);
@@ -314,9 +298,13 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ------------------------------------------------------------------ softmax / epilogue
         // A failed (timed-out) wait sets `fail`; the four warps learn it at the
         // next named barrier of the group and leave the loop together.
+        // S rows live in lanes 0..15 of each TMEM quadrant (M = 64 layout); lane l + 16 takes
+        // tokens 32..63 of the head of lane l, received by shuffles.
         const int qd = warp & 3;                 // TMEM lane quadrant
-        const int h = 16 * qd + lane;            // head row of S owned by this thread (lane < 16)
-        const bool head = lane < 16 && h < HQ;
+        const int half = lane >> 4;              // 0: tokens 0..31 of the tile, 1: tokens 32..63
+        const int h = 16 * qd + (lane & 15);     // head
+        const bool head = h < HQ;
+        const int base = 32 * half;
         const int tid = threadIdx.x - 64;        // 0..127
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
         uint32_t seq = 0, unit_k = 0;
@@ -360,25 +348,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!fail) fail = !mbar_wait(bar + B_S_FULL + ts, par, s_abort, a.status);
             if (threadIdx.x == 64) TRACE(6, seq);
             umma::fence_after_sync();
-            uint32_t sr[kT];
-            umma::ld32(t_s + lane_off + ts * kT, *reinterpret_cast<uint32_t(*)[32]>(sr));
-            umma::ld32(t_s + lane_off + ts * kT + 32, *reinterpret_cast<uint32_t(*)[32]>(sr + 32));
-            umma::wait_ld();
-            float alpha = 1.f;
-            if (head) {
-                float mt = -INFINITY;
+            float x[32];
+            {
+                uint32_t v0[32], v1[32];
+                umma::ld32(t_s + lane_off + ts * kT, v0);
+                umma::ld32(t_s + lane_off + ts * kT + 32, v1);
+                umma::wait_ld();
 #pragma unroll
-                for (int j = 0; j < kT; j++) {
-                    const float v = j < nvalid ? __uint_as_float(sr[j]) * a.scale_log2 : -INFINITY;
-                    sr[j] = __float_as_uint(v);
-                    mt = fmaxf(mt, v);
+                for (int j = 0; j < 32; j++) {
+                    const uint32_t recv = __shfl_xor_sync(0xffffffffu, v1[j], 16);
+                    const float v = __uint_as_float(half ? recv : v0[j]);
+                    x[j] = base + j < nvalid ? v * a.scale_log2 : -INFINITY;
                 }
-                if (mt > m_used + kRescaleLog2 || (m_used == -INFINITY && mt != -INFINITY)) {
-                    alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - mt);
-                    m_used = mt;
-                }
-                s_alpha[h] = alpha;
             }
+            float mt = -INFINITY;
+#pragma unroll
+            for (int j = 0; j < 32; j++) mt = fmaxf(mt, x[j]);
+            mt = fmaxf(mt, __shfl_xor_sync(0xffffffffu, mt, 16));
+            float alpha = 1.f;
+            if (mt > m_used + kRescaleLog2 || (m_used == -INFINITY && mt != -INFINITY)) {
+                alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - mt);
+                m_used = mt;
+            }
+            if (head && half == 0) s_alpha[h] = alpha;
             if (threadIdx.x == 64) TRACE(7, seq);
             // one barrier: some head rescaled while O^T holds data, or a wait failed (a failing
             // thread republishes the abort flag first, so every thread reads it set after the barrier)
@@ -410,10 +402,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             // read it), P_lo into its buffer
             if (!fail && head) {
                 float rowsum = 0.f;
-                uint32_t phw[kT / 2], plw[kT / 2];
+                uint32_t phw[16], plw[16];
 #pragma unroll
-                for (int j = 0; j < kT; j += 2) {
-                    const float x0 = __uint_as_float(sr[j]), x1 = __uint_as_float(sr[j + 1]);
+                for (int j = 0; j < 32; j += 2) {
+                    const float x0 = x[j], x1 = x[j + 1];
                     const float p0 = x0 == -INFINITY ? 0.f : fast_exp2(x0 - m_used);
                     const float p1 = x1 == -INFINITY ? 0.f : fast_exp2(x1 - m_used);
                     rowsum += p0 + p1;
@@ -426,12 +418,14 @@ __global__ void __launch_bounds__(kThreads, 1)
                 lsum = lsum * alpha + rowsum;
                 uint8_t* prow = sm + kOffTiles + (size_t)ts * kTileBytes + 8 * kBox;
                 uint8_t* lrow = sm + kOffPlo;
+                // my 32 tokens = 16-byte chunks 4 half .. 4 half + 3 of row h
 #pragma unroll
-                for (int c = 0; c < 8; c++) {
+                for (int cc = 0; cc < 4; cc++) {
+                    const int c = 4 * half + cc;
                     *reinterpret_cast<uint4*>(prow + sw128(h, c)) =
-                        make_uint4(phw[4 * c], phw[4 * c + 1], phw[4 * c + 2], phw[4 * c + 3]);
+                        make_uint4(phw[4 * cc], phw[4 * cc + 1], phw[4 * cc + 2], phw[4 * cc + 3]);
                     *reinterpret_cast<uint4*>(lrow + sw128(h, c)) =
-                        make_uint4(plw[4 * c], plw[4 * c + 1], plw[4 * c + 2], plw[4 * c + 3]);
+                        make_uint4(plw[4 * cc], plw[4 * cc + 1], plw[4 * cc + 2], plw[4 * cc + 3]);
                 }
             }
             if (!fail && nvalid < kT) {
@@ -456,7 +450,8 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (last) {
                 if (!fail) fail = !mbar_wait(bar + B_PV_DONE + ts, par, s_abort, a.status);
                 umma::fence_after_sync();
-                if (head) s_l[h] = lsum > 0.f ? 1.f / lsum : 0.f;  // O = O^T * (1 / l)
+                const float l = lsum + __shfl_xor_sync(0xffffffffu, lsum, 16);  // both halves of the head
+                if (head && half == 0) s_l[h] = l > 0.f ? 1.f / l : 0.f;      // O = O^T * (1 / l)
                 if (named_barrier_or(kSmBar, 128, fail)) break;
                 const int64_t shard = (int64_t)u.n * a.batch + u.b;
                 const bool split = u.n_chunks > 1;
@@ -475,7 +470,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                             __stcg(obase + (int64_t)(c0 + i) * 512 + dv, __uint_as_float(r[i]) * s_l[c0 + i]);
                     }
                 }
-                if (head) __stcg(lbase + h, lsum > 0.f ? (m_used + log2f(lsum)) * kLn2 : -INFINITY);
+                if (head && half == 0) __stcg(lbase + h, l > 0.f ? (m_used + log2f(l)) * kLn2 : -INFINITY);
                 umma::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar + B_O_FREE);
