@@ -10,9 +10,10 @@
 // 6.5 TB/s, beyond the CUDA-core fp32 rate but far below the tensor pipe, so
 // the kernel is HBM-bound and uses warp-level mma.sync m16n8k16 (fp32
 // accumulate): the 16 heads of a KV head fill M exactly, tokens are N.  Q K^T
-// runs in bf16 (exact products); P V runs in f16 so that P keeps 11
-// significant bits (V fragments are widened in registers, saturating at
-// +-65504).
+// runs in bf16 (exact products); P V runs in bf16 on the V fragments as loaded,
+// with P split into two bf16 terms (P_hi + P_lo, 16 significant bits).  The
+// running maximum is rescaled lazily: only when a row's maximum grows by more
+// than 2^8, so the 16 x D accumulator is rarely touched.
 //
 // Structure: persistent grid, one work unit (shard, request, chunk) per CTA
 // iteration, all KV heads in the CTA.  Warp NCW (producer) issues TMA tiled
@@ -32,6 +33,7 @@ namespace dcp {
 namespace {
 
 constexpr int kTok = 16;            // tokens per stage
+constexpr float kRescaleLog2 = 8.f;  // lazy rescale threshold (log2 units)
 constexpr int kBoxBytes = kTok * 128;  // one [16][64] bf16 box (128-byte rows)
 
 __device__ __forceinline__ void ldsm_x4(uint32_t addr, uint32_t& r0, uint32_t& r1, uint32_t& r2, uint32_t& r3) {
@@ -54,24 +56,13 @@ __device__ __forceinline__ void mma_bf16(float* d, const uint32_t* a, uint32_t b
         : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
 }
 
-__device__ __forceinline__ void mma_f16(float* d, const uint32_t* a, uint32_t b0, uint32_t b1) {
-    asm volatile(
-        "mma.sync.aligned.m16n8k16.row.col.f32.f16.f16.f32 {%0, %1, %2, %3}, {%4, %5, %6, %7}, {%8, %9}, "
-        "{%0, %1, %2, %3};"
-        : "+f"(d[0]), "+f"(d[1]), "+f"(d[2]), "+f"(d[3])
-        : "r"(a[0]), "r"(a[1]), "r"(a[2]), "r"(a[3]), "r"(b0), "r"(b1));
-}
-
-__device__ __forceinline__ uint32_t pack_f16(float lo, float hi) {
-    __half2 v = __floats2half2_rn(lo, hi);
-    return *reinterpret_cast<uint32_t*>(&v);
-}
-
-// two bf16 (one 32-bit register) -> two f16, saturating at +-65504
-__device__ __forceinline__ uint32_t bf16x2_to_f16x2(uint32_t w) {
-    const float lo = fminf(fmaxf(__uint_as_float(w << 16), -65504.f), 65504.f);
-    const float hi = fminf(fmaxf(__uint_as_float(w & 0xFFFF0000u), -65504.f), 65504.f);
-    return pack_f16(lo, hi);
+// two floats -> bf16x2 high terms and bf16x2 residuals (x0 ~ hi.x + lo.x, x1 ~ hi.y + lo.y)
+__device__ __forceinline__ void split_bf16(float x0, float x1, uint32_t& hi, uint32_t& lo) {
+    const __nv_bfloat162 h = __floats2bfloat162_rn(x0, x1);
+    const float2 hf = __bfloat1622float2(h);
+    const __nv_bfloat162 l = __floats2bfloat162_rn(x0 - hf.x, x1 - hf.y);
+    hi = *reinterpret_cast<const uint32_t*>(&h);
+    lo = *reinterpret_cast<const uint32_t*>(&l);
 }
 
 // byte offset of (row r, column c) inside one [16][64] bf16 box with 128-byte swizzle
@@ -255,10 +246,18 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
                 mx0 = fmaxf(mx0, __shfl_xor_sync(0xffffffffu, mx0, 2));
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 1));
                 mx1 = fmaxf(mx1, __shfl_xor_sync(0xffffffffu, mx1, 2));
-                const float mn0 = fmaxf(m0, mx0), mn1 = fmaxf(m1, mx1);
-                const float c0 = fast_exp2(m0 - mn0), c1 = fast_exp2(m1 - mn1);
-                m0 = mn0;
-                m1 = mn1;
+                // lazy rescale: the reference maximum moves only when a row's maximum grows by
+                // more than 2^8 (p stays <= 2^8), so O is rarely rescaled
+                float c0 = 1.f, c1 = 1.f;
+                if (mx0 > m0 + kRescaleLog2 || (m0 == -INFINITY && mx0 != -INFINITY)) {
+                    c0 = m0 == -INFINITY ? 0.f : fast_exp2(m0 - mx0);
+                    m0 = mx0;
+                }
+                if (mx1 > m1 + kRescaleLog2 || (m1 == -INFINITY && mx1 != -INFINITY)) {
+                    c1 = m1 == -INFINITY ? 0.f : fast_exp2(m1 - mx1);
+                    m1 = mx1;
+                }
+                const float mn0 = m0 == -INFINITY ? 0.f : m0, mn1 = m1 == -INFINITY ? 0.f : m1;
                 float p[2][4];
 #pragma unroll
                 for (int nt = 0; nt < 2; nt++) {
@@ -269,16 +268,21 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
                 }
                 l0 = l0 * c0 + p[0][0] + p[0][1] + p[1][0] + p[1][1];
                 l1 = l1 * c1 + p[0][2] + p[0][3] + p[1][2] + p[1][3];
+                if (c0 != 1.f || c1 != 1.f) {
 #pragma unroll
-                for (int i = 0; i < D / 8; i++) {
-                    o[i][0] *= c0;
-                    o[i][1] *= c0;
-                    o[i][2] *= c1;
-                    o[i][3] *= c1;
+                    for (int i = 0; i < D / 8; i++) {
+                        o[i][0] *= c0;
+                        o[i][1] *= c0;
+                        o[i][2] *= c1;
+                        o[i][3] *= c1;
+                    }
                 }
-                // P V in f16 (11 significant bits for P): V fragments are widened in registers
-                uint32_t pa[4] = {pack_f16(p[0][0], p[0][1]), pack_f16(p[0][2], p[0][3]),
-                                  pack_f16(p[1][0], p[1][1]), pack_f16(p[1][2], p[1][3])};
+                // P V in bf16 with P = P_hi + P_lo (16 significant bits), V fragments as loaded
+                uint32_t pa[4], pl[4];
+                split_bf16(p[0][0], p[0][1], pa[0], pl[0]);
+                split_bf16(p[0][2], p[0][3], pa[1], pl[1]);
+                split_bf16(p[1][0], p[1][1], pa[2], pl[2]);
+                split_bf16(p[1][2], p[1][3], pa[3], pl[3]);
                 // rows past the unit's last token hold stale page contents: zero them so that
                 // P = 0 cannot meet a NaN/Inf in the P V product
                 if (nvalid < kTok) {
@@ -300,8 +304,10 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
                     const uint32_t addr = vbase + (uint32_t)(col / 64) * kBoxBytes + swz(tok, col & 63);
                     uint32_t b0, b1, b2, b3;
                     ldsm_x4_t(addr, b0, b1, b2, b3);
-                    mma_f16(o[jn], pa, bf16x2_to_f16x2(b0), bf16x2_to_f16x2(b1));
-                    mma_f16(o[jn + 1], pa, bf16x2_to_f16x2(b2), bf16x2_to_f16x2(b3));
+                    mma_bf16(o[jn], pa, b0, b1);
+                    mma_bf16(o[jn + 1], pa, b2, b3);
+                    mma_bf16(o[jn], pl, b0, b1);
+                    mma_bf16(o[jn + 1], pl, b2, b3);
                 }
             }
         }
