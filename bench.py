@@ -58,6 +58,8 @@ def parse():
     ap.add_argument("--batch-limit", type=int, default=None,
                     help="keep only the first B requests of the workload (small profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--bands", action="store_true",
+                    help="also time the decode per request-length band (<32k, 32-64k, 64-128k, 128-200k, 200k+)")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=25.0, help="target CPU work of the oracle sample")
     return ap.parse_args()
@@ -210,6 +212,36 @@ def combine_ranks(dist, device, ms, kern_total, e2e_ms, bytes_timed, e2e_bytes):
 # our implementation
 # ----------------------------------------------------------------------------
 
+BANDS = [(0, 32_000, "<32k"), (32_000, 64_000, "32-64k"), (64_000, 128_000, "64-128k"),
+         (128_000, 200_000, "128-200k"), (200_000, 1 << 31, "200k+")]
+
+
+def time_bands(args, w, dcp, dw, q, lens, o_part, lse, stream, reps: int = 5):
+    """Decode time per request-length band: the other requests get length 0 (their
+    shards are empty), so the launch covers exactly the band's tokens."""
+    import torch
+    out = {}
+    L = lens.cpu().numpy()
+    for lo, hi, name in BANDS:
+        sel = (L >= lo) & (L < hi)
+        if not sel.any():
+            continue
+        lb = torch.as_tensor(np.where(sel, L, 0).astype(np.int32), device=lens.device)
+        for _ in range(2):
+            dcp.dcp_decode_partial(dw.desc, q, lb, o_part, lse, dw.ws)
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            dcp.dcp_decode_partial(dw.desc, q, lb, o_part, lse, dw.ws)
+        e1.record(stream)
+        torch.cuda.synchronize()
+        ms = e0.elapsed_time(e1) / reps
+        tok = int(L[sel].sum())
+        out[name] = {"requests": int(sel.sum()), "tokens": tok, "decode_ms": round(ms, 4),
+                     "kv_gbs": round(tok * w.kv_bytes_per_token / (ms * 1e-3) / 1e9, 1)}
+    return out
+
+
 def run_ours(args, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -296,6 +328,9 @@ def run_ours(args, rank, world, local_rank):
     ms = t_start.elapsed_time(t_stop)
     kern_ms = [a.elapsed_time(b) for a, b in ev_k]
     bytes_timed = sum(kv_tok[args.warmup + i] for i in range(args.steps)) * bpt
+
+    bands = time_bands(args, w, dcp, dw, qs[args.warmup], lens_s[args.warmup], o_part, lse, stream) \
+        if args.bands else None
 
     # end to end through the C ABI with host buffers: H2D of the step's inputs
     # (q, new token rows, positions, lengths) from pinned memory, D2H of out + lse
@@ -384,6 +419,8 @@ def run_ours(args, rank, world, local_rank):
         "gpu_launches": launches_per_step(w) * args.steps,
         "fill_seconds": round(fill_s, 2),
     }
+    if bands is not None:
+        res["bands"] = bands
     if e2e:
         res["e2e"] = {"value": round(e2e_bytes_all / (e2e_ms_max * 1e-3) / 1e9, 1), "unit": "GB/s",
                       "h2d_bytes_per_step": e2e[2], "d2h_bytes_per_step": e2e[3],
@@ -408,11 +445,11 @@ def oracle_sample(w, cpu_seconds: float, q64):
     shortest request is timed first and the rate extrapolated (conservatively:
     more requests run more parallel work items)."""
     order = [int(b) for b in np.argsort(synth.bits(synth.key(w.seed_len, 7), np.arange(w.B)))]
-    probe = min(order, key=lambda b: int(w.lengths[b]))
+    probe = sorted(order, key=lambda b: int(w.lengths[b]))[:4]  # enough work items for the threads
     t0 = time.perf_counter()
-    _oracle_run(w, q64, [probe])
-    rate = max(1.0, int(w.lengths[probe])) / max(time.perf_counter() - t0, 1e-4)  # tokens per second
-    budget_tok = max(int(w.lengths[probe]), int(cpu_seconds * rate))
+    _oracle_run(w, q64, probe)
+    rate = max(1.0, float(sum(int(w.lengths[b]) for b in probe))) / max(time.perf_counter() - t0, 1e-4)
+    budget_tok = max(int(min(w.lengths)), int(cpu_seconds * rate))
     reqs, tot = [], 0
     for b in order:
         if tot + int(w.lengths[b]) > budget_tok and reqs:
