@@ -87,7 +87,6 @@ constexpr int kPPage = 2 * kPTerm;         // both terms of one page
 constexpr int kPBuf = 2 * kPPage;          // a tile of two pages: 16 KB
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kSmBar = 1;                  // the 256 softmax threads
-constexpr int kPairBar = 2;                // + quadrant: the two warps sharing a TMEM lane quadrant
 constexpr int kSoftWarps = 8;
 constexpr int kThreads = 32 * (3 + kSoftWarps);  // producer, S issuer, softmax x 8, P V issuer
 constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384;  // TMEM columns
@@ -99,8 +98,8 @@ constexpr uint32_t kOffScales = kOffP + 2 * kPBuf;
 constexpr uint32_t kOffBars = kOffScales + kSlots * kPg * 4;
 constexpr uint32_t kOffMeta = kOffBars + 32 * 8;
 constexpr uint32_t kOffSmall = kOffMeta + kSlots * 16;
-// s_alpha[64], s_inv[64], s_gmax[2][64], s_gsmax[2][64], s_gl[2][64], misc[16]
-constexpr uint32_t kSmemBytes = kOffSmall + (8 * 64 + 16) * 4 + 1024;
+// s_alpha[64], s_inv[64], s_gmax[2][64], s_gl[2][64], misc[16]
+constexpr uint32_t kSmemBytes = kOffSmall + (6 * 64 + 16) * 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
 static_assert(kOffRope % 1024 == 0 && kOffP % 1024 == 0, "swizzled operands need 1 KB alignment");
 
@@ -244,9 +243,8 @@ __global__ void __launch_bounds__(kThreads, 1)
     StageMeta* tmeta = reinterpret_cast<StageMeta*>(sm + kOffMeta);  // per page slot
     float* s_alpha = reinterpret_cast<float*>(sm + kOffSmall);
     float* s_inv = s_alpha + 64;
-    float* s_gmax = s_inv + 64;     // [2 token groups][64 heads]
-    float* s_gsmax = s_gmax + 128;  // [2][64]
-    float* s_gl = s_gsmax + 128;    // [2][64]
+    float* s_gmax = s_inv + 64;     // [2 pages][64 heads]: each page's bound on x + log2 s
+    float* s_gl = s_gmax + 128;     // [2][64]
     int* s_misc = reinterpret_cast<int*>(s_gl + 128);  // [0] tmem base, [2] split flag, [3] abort
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_misc + 3);
 
@@ -590,30 +588,29 @@ __global__ void __launch_bounds__(kThreads, 1)
             for (int j = 0; j < 32; j++) mx = fmaxf(mx, x[j]);
             mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, 16));
             smax = fmaxf(smax, __shfl_xor_sync(0xffffffffu, smax, 16));
-            // combine with the other page of the tile (same heads)
-            if (half == 0) {
-                s_gmax[wg * 64 + h] = mx;
-                s_gsmax[wg * 64 + h] = smax;
-            }
-            named_barrier_sync(kPairBar + qd, 64);
-            mx = fmaxf(mx, s_gmax[(wg ^ 1) * 64 + h]);
-            smax = fmaxf(smax, s_gsmax[(wg ^ 1) * 64 + h]);
-            // m >= max_t (x_t + log2 s_t): the weights 2^(x - m) s_t stay <= 2^8
-            const float mt = (mx == -INFINITY || !(smax > 0.f)) ? mx : mx + __log2f(smax);
+            // Bound of this page: m_g = max_t x_t + log2 max_t s_t >= x_t + log2 s_t for its tokens;
+            // the tile's bound is the larger of the two pages' (the weights 2^(x - m) s_t stay <= 2^8).
+            // A head's running maximum moves iff one of its pages' bounds passes the threshold, so
+            // one barrier both exchanges the bounds and decides whether any head rescales.
+            const float mt_g = (mx == -INFINITY || !(smax > 0.f)) ? mx : mx + __log2f(smax);
+            if (half == 0) s_gmax[wg * 64 + h] = mt_g;
+            const bool moves = mt_g > m_used + kRescaleLog2 || (m_used == -INFINITY && mt_g != -INFINITY);
+            if (threadIdx.x == 64) TRACE(7, seq);
+            // (a failing thread republishes the abort flag first, so every thread reads it set after
+            // the barrier)
+            if (fail) *s_abort = 1;
+            const int any = named_barrier_or(kSmBar, 256, fail || (head && moves && o_has));
+            if (any && *s_abort) break;
+            const float mt = fmaxf(mt_g, s_gmax[(wg ^ 1) * 64 + h]);
             float alpha = 1.f;
             if (mt > m_used + kRescaleLog2 || (m_used == -INFINITY && mt != -INFINITY)) {
                 alpha = (m_used == -INFINITY) ? 0.f : fast_exp2(m_used - mt);
                 m_used = mt;
             }
-            if (half == 0 && wg == 0) s_alpha[h] = alpha;
-            if (threadIdx.x == 64) TRACE(7, seq);
-            // one barrier: some head rescaled while O^T holds data, or a wait failed (a failing
-            // thread republishes the abort flag first, so every thread reads it set after the barrier)
-            if (fail) *s_abort = 1;
-            const int any = named_barrier_or(kSmBar, 256, fail || (head && alpha != 1.f && o_has));
-            if (any && *s_abort) break;
             if (threadIdx.x == 64) TRACE(8, seq);
             if (any) {
+                if (half == 0 && wg == 0) s_alpha[h] = alpha;
+                named_barrier_sync(kSmBar, 256);
                 // the previous tile's P V must be complete before O^T is rescaled; token group wg
                 // rescales value blocks 2 wg, 2 wg + 1 of its lane quadrant
                 fail = !mbar_wait(bar + B_PV_DONE + (pb ^ 1), ((seq - 1) >> 1) & 1, s_abort, a.status);
