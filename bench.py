@@ -166,10 +166,11 @@ KERNEL_SOURCES = os.path.join(ROOT, "sequence_sharded_paged_b200", "csrc")
 
 
 def kernel_sources_digest() -> str:
-    """sha256 over the CUDA sources of the library (a changed kernel voids old counters)."""
+    """sha256 over the sources of what the decode launch runs: the planner, the decode
+    kernels and the headers they include (a changed kernel voids old counters)."""
     h = hashlib.sha256()
     for name in sorted(os.listdir(KERNEL_SOURCES)):
-        if name.endswith((".cu", ".cuh", ".h")):
+        if name == "plan.cu" or name.startswith("decode_") or name.endswith((".cuh", ".h")) or name == "tma.cu":
             h.update(name.encode())
             h.update(open(os.path.join(KERNEL_SOURCES, name), "rb").read())
     return h.hexdigest()

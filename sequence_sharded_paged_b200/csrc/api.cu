@@ -132,8 +132,8 @@ bool make_plan_within(const dcp_cache_desc* c, int B, int num_sms, size_t cap, P
     return p->lay.total <= cap;
 }
 
-// The launch sequence of dcp_decode_partial (plan kernel, decode kernel) on a
-// workspace `w` laid out by `p`.
+// The launch sequence of the decode (plan kernel, decode kernel) on a workspace
+// `w` laid out by `p`.
 dcp_status decode_on(const dcp_cache_desc* cache, int32_t B, const void* q, const int32_t* seq_lens,
                      float* o_partial, float* lse, uint8_t* w, const Plan& p, int* status, cudaStream_t s) {
     const int64_t target = (int64_t)p.g.units_per_cta * p.g.ctas;
@@ -348,45 +348,7 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
     Plan p;
     if (!make_plan(cache, B, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
     if (ws_bytes < p.lay.total) return DCP_ERR_WORKSPACE_TOO_SMALL;
-    cudaStream_t s = (cudaStream_t)stream;
-    uint8_t* w = static_cast<uint8_t*>(ws);
-    const int64_t target = (int64_t)p.g.units_per_cta * p.g.ctas;
-    cudaError_t e = launch_plan(seq_lens, B, cache->n_shards, cache->interleave, p.g.granule, p.g.min_chunk,
-                                (int)target, p.g.n_hb, ws, p.lay.max_units, p.lay.max_split, cache->hq, cache->dv,
-                                status, s);
-    if (e != cudaSuccess) return DCP_ERR_CUDA;
-    DecodeArgs a;
-    a.k_pages = static_cast<const uint8_t*>(cache->k_pages);
-    a.v_pages = static_cast<const uint8_t*>(cache->v_pages);
-    a.kv_scales = cache->dtype == DCP_FP8_E4M3 ? cache->kv_scales : nullptr;
-    a.block_tables = cache->block_tables;
-    a.n_shards = cache->n_shards;
-    a.interleave = cache->interleave;
-    a.page_size = cache->page_size;
-    a.num_pages = cache->num_pages;
-    a.batch = B;
-    a.max_local_pages = cache->max_local_pages;
-    a.hq = cache->hq;
-    a.hkv = cache->hkv;
-    a.dk = cache->dk;
-    a.dv = cache->dv;
-    a.scale_log2 = cache->scale * kLog2e;
-    a.q = static_cast<const __nv_bfloat16*>(q);
-    a.seq_lens = seq_lens;
-    a.o_partial = o_partial;
-    a.lse = lse;
-    a.plan = reinterpret_cast<const PlanHeader*>(w);
-    a.ticket = &reinterpret_cast<PlanHeader*>(w)->next_unit;
-    a.units = reinterpret_cast<const Unit*>(w + p.lay.off_units);
-    a.done = reinterpret_cast<int32_t*>(w + p.lay.off_done);
-    a.split_o = reinterpret_cast<float*>(w + p.lay.off_split_o);
-    a.split_lse = reinterpret_cast<float*>(w + p.lay.off_split_lse);
-    a.qs = p.off_qs ? w + p.off_qs : nullptr;
-    a.qinv = p.off_qinv ? reinterpret_cast<float*>(w + p.off_qinv) : nullptr;
-    a.status = status;
-    e = launch_decode(p.g, a, s);
-    if (e == cudaErrorNotSupported) return DCP_ERR_UNSUPPORTED;
-    return cuda_err(e);
+    return decode_on(cache, B, q, seq_lens, o_partial, lse, static_cast<uint8_t*>(ws), p, status, (cudaStream_t)stream);
 }
 
 // No workspace argument and no allocation: for callers that cannot allocate
