@@ -165,12 +165,21 @@ TRAFFIC_FILE = os.path.join(ROOT, "profiles", "decode_dram_traffic.json")
 KERNEL_SOURCES = os.path.join(ROOT, "sequence_sharded_paged_b200", "csrc")
 
 
-def kernel_sources_digest() -> str:
-    """sha256 over the sources of what the decode launch runs: the planner, the decode
-    kernels and the headers they include (a changed kernel voids old counters)."""
+# the decode kernel of each capture and the source file it is built from
+KERNEL_FILES = {"gqa_mma_kernel": "decode_gqa_mma.cu", "mla_bf16_kernel": "decode_mla_bf16.cu",
+                "mla_fp8_kernel": "decode_mla_fp8.cu", "gqa_simt_kernel": "decode_simt.cu",
+                "mla_simt_kernel": "decode_simt.cu"}
+
+
+def kernel_sources_digest(kernel: str) -> str:
+    """sha256 over the sources that one decode kernel is built from: the planner, the
+    tensor-map code, the shared headers and the kernel's own file. A change to any of
+    them voids the counters captured for that kernel; a change to another decode
+    kernel does not."""
+    own = KERNEL_FILES[kernel.split("<")[0]]
     h = hashlib.sha256()
     for name in sorted(os.listdir(KERNEL_SOURCES)):
-        if name == "plan.cu" or name.startswith("decode_") or name.endswith((".cuh", ".h")) or name == "tma.cu":
+        if name in ("plan.cu", "tma.cu", own) or name.endswith((".cuh", ".h")):
             h.update(name.encode())
             h.update(open(os.path.join(KERNEL_SOURCES, name), "rb").read())
     return h.hexdigest()
@@ -178,14 +187,13 @@ def kernel_sources_digest() -> str:
 
 def measured_traffic(config_key: str):
     """dram bytes read + written per decode launch, or None when no capture of
-    the current sources exists for this workload."""
+    the current sources of that workload's decode kernel exists."""
     if not os.path.exists(TRAFFIC_FILE):
         return None
-    d = json.load(open(TRAFFIC_FILE))
-    if d.get("sources_sha256") != kernel_sources_digest():
+    e = json.load(open(TRAFFIC_FILE)).get("workloads", {}).get(config_key)
+    if e is None or e.get("sources_sha256") != kernel_sources_digest(e["kernel"]):
         return None
-    e = d.get("workloads", {}).get(config_key)
-    return None if e is None else float(e["dram_bytes_per_launch"])
+    return float(e["dram_bytes_per_launch"])
 
 
 def traffic_key(args, w) -> str:

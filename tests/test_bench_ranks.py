@@ -1,5 +1,6 @@
 """Host-side logic of bench.py: the multi-rank reduction (max of device time,
-sum of bytes) on two gloo ranks, and the clock-sample summary."""
+sum of bytes) on two gloo ranks, the clock-sample summary, and which source
+changes void a stored DRAM-traffic capture."""
 from __future__ import annotations
 
 import os
@@ -75,3 +76,36 @@ def test_launch_count_per_path():
     assert bench.launches_per_step(synth.workload(5)) == 6   # fp8 MLA: + query split
     assert bench.launches_per_step(synth.workload(4)) == 5
     assert bench.launches_per_step(synth.workload(3)) == 5
+
+
+def test_traffic_digest_is_per_kernel(tmp_path, monkeypatch):
+    """Editing one decode kernel's file voids that kernel's counters only; a shared
+    header voids them all."""
+    import shutil
+    src = tmp_path / "csrc"
+    shutil.copytree(bench.KERNEL_SOURCES, src)
+    monkeypatch.setattr(bench, "KERNEL_SOURCES", str(src))
+    kernels = ["gqa_mma_kernel<128,4>", "mla_bf16_kernel<64>", "mla_fp8_kernel<64>"]
+    before = {k: bench.kernel_sources_digest(k) for k in kernels}
+    with open(src / "decode_mla_fp8.cu", "a") as f:
+        f.write("\n// edited\n")
+    after = {k: bench.kernel_sources_digest(k) for k in kernels}
+    assert after["mla_fp8_kernel<64>"] != before["mla_fp8_kernel<64>"]
+    assert after["gqa_mma_kernel<128,4>"] == before["gqa_mma_kernel<128,4>"]
+    assert after["mla_bf16_kernel<64>"] == before["mla_bf16_kernel<64>"]
+    with open(src / "common.cuh", "a") as f:
+        f.write("\n// edited\n")
+    shared = {k: bench.kernel_sources_digest(k) for k in kernels}
+    assert all(shared[k] != after[k] for k in kernels)
+
+
+def test_committed_traffic_file_is_well_formed():
+    """Each capture names a known decode kernel, carries its sources' digest, and reads
+    no fewer bytes than the launch's KV cache."""
+    import json
+    d = json.load(open(bench.TRAFFIC_FILE))
+    for key, e in d["workloads"].items():
+        assert e["kernel"].split("<")[0] in bench.KERNEL_FILES, key
+        assert len(e["sources_sha256"]) == 64, key
+        assert abs(e["dram_read"] + e["dram_write"] - e["dram_bytes_per_launch"]) < 1e3, key
+        assert 0.99 < e["dram_bytes_per_launch"] / e["algorithmic_kv_bytes"] < 1.3, key
