@@ -181,7 +181,20 @@ size_t dcp_decode_workspace_size(const dcp_cache_desc* cache, int32_t B);
  *             -inf when it owns none.
  *  ws, ws_bytes  device workspace of at least dcp_decode_workspace_size()
  *             bytes; its contents need no initialisation and are clobbered.
- * Concurrent calls must use distinct workspaces.
+ * Concurrent calls must use distinct workspaces.  The work is queued on
+ * `stream`; the call does not wait for it.
+ * Errors, returned before anything is launched:
+ *  DCP_ERR_INVALID_ARG     a bad descriptor, B != cache->batch, or a NULL pointer;
+ *  DCP_ERR_MISALIGNED      q, o_partial, lse, ws or a pool not 16-byte aligned;
+ *  DCP_ERR_UNSUPPORTED     a shape no kernel of this build covers (page size,
+ *                          head size, group size);
+ *  DCP_ERR_WORKSPACE_TOO_SMALL  ws_bytes below dcp_decode_workspace_size();
+ *  DCP_ERR_CUDA            a launch or an attribute call failed.
+ * Device-side errors, read with dcp_get_device_status:
+ *  DCP_ERR_UNALLOCATED_PAGE  an attended position's page is not a pool page; its
+ *                          tokens are skipped;
+ *  DCP_ERR_TIMEOUT         a kernel gave up waiting on a copy; the outputs of that
+ *                          call are then unspecified.
  */
 dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void* q, const int32_t* seq_lens,
                               float* o_partial, float* lse, void* ws, size_t ws_bytes, void* stream);
