@@ -1,6 +1,7 @@
 """Host-side logic of bench.py: the multi-rank reduction (max of device time,
-sum of bytes) on two gloo ranks, the clock-sample summary, and which source
-changes void a stored DRAM-traffic capture."""
+sum of bytes) on two gloo ranks, the clock-sample summary, which source changes
+void a stored DRAM-traffic capture, and the reference arm's JSON line (the oracle
+on host cores)."""
 from __future__ import annotations
 
 import os
@@ -109,3 +110,33 @@ def test_committed_traffic_file_is_well_formed():
         assert len(e["sources_sha256"]) == 64, key
         assert abs(e["dram_read"] + e["dram_write"] - e["dram_bytes_per_launch"]) < 1e3, key
         assert 0.99 < e["dram_bytes_per_launch"] / e["algorithmic_kv_bytes"] < 1.3, key
+
+
+def _bench_reference(env_extra):
+    import json
+    import subprocess
+    env = dict(os.environ, **env_extra)
+    r = subprocess.run([sys.executable, os.path.join(ROOT, "bench.py"), "--impl", "reference", "--config", "1",
+                        "--steps", "2", "--warmup", "1"], capture_output=True, text=True, env=env, timeout=600,
+                       cwd=ROOT)
+    assert r.returncode == 0, r.stderr[-2000:]
+    lines = [l for l in r.stdout.splitlines() if l.strip()]
+    return [json.loads(l) for l in lines]
+
+
+def test_reference_arm_json_line():
+    """The reference arm (the oracle on host cores) prints one JSON line with the bench contract's keys."""
+    (d,) = _bench_reference({"WORLD_SIZE": "1", "RANK": "0"})
+    assert d["impl"] == "reference" and d["metric"] == bench.METRIC and d["unit"] == "GB/s"
+    assert d["value"] > 0 and d["ms_per_step"] > 0
+    assert (d["n_gpus"], d["steps"], d["warmup"]) == (1, 2, 1)
+    assert d["higher_is_better"] is True and d["scaling"] == "weak" and d["vs_baseline"] is None
+    assert d["dtype"] == "f64" and "synthetic" in d["data"] and "workload" in d["config"]
+    cb = d["cpu_baseline"]
+    assert cb["kind"] == "oracle" and cb["cores"] >= 1 and cb["sample"] and cb["value"] == d["value"]
+    assert d["e2e"] == {"value": d["value"], "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}
+
+
+def test_reference_arm_other_ranks_are_silent():
+    """Under torchrun only rank 0 runs the oracle and prints; the other ranks exit 0 without output."""
+    assert _bench_reference({"WORLD_SIZE": "2", "RANK": "1"}) == []
