@@ -15,7 +15,7 @@ import synth
 import synth.device as sdev
 from sequence_sharded_paged_b200 import workload as wl
 
-from gpu_util import (TOL_LSE, build_for_test, compare, oracle_decode, run_step, small_workload, vmax_attended)
+from gpu_util import (build_for_test, compare, oracle_decode, run_step, small_workload, vmax_attended)
 
 pytestmark = pytest.mark.gpu
 

@@ -6,7 +6,6 @@ import re
 import subprocess
 import tempfile
 
-import pytest
 
 import sequence_sharded_paged_b200 as dcp
 import synth

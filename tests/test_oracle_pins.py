@@ -9,7 +9,6 @@ operand, an off-by-one in the local packing) fails at least one of them.
 import json
 import math
 import os
-from fractions import Fraction
 
 import numpy as np
 import pytest
