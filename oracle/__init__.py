@@ -93,6 +93,9 @@ def lib():
         L.orc_decode.argtypes = [ctypes.POINTER(_Cache), P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
                                  P, ctypes.c_int32, P, P]
         L.orc_decode.restype = ctypes.c_int
+        L.orc_decode_multi.argtypes = [ctypes.POINTER(_Cache), P, P, ctypes.c_int32, ctypes.c_int32, ctypes.c_int32,
+                                       ctypes.c_int32, P, P]
+        L.orc_decode_multi.restype = ctypes.c_int
         L.orc_merge.argtypes = [ctypes.c_int32] * 4 + [P] * 4
         L.orc_merge.restype = None
         L.orc_synth_bf16.argtypes = [ctypes.c_uint64, ctypes.c_uint64, ctypes.c_int64, P, P]
@@ -231,6 +234,40 @@ def decode_synth(kind: str, dtype: str, seed: int, q, seq_lens, scale: float, hk
     c = _Cache(1 if kind == "mla" else 0, 1 if dtype == "fp8" else 0, B, Hq, hkv, dk, dv, scale, 1, None, None,
                0, seed)
     return _decode(c, q, seq_lens, N, I, shard, req_list)
+
+
+def _decode_multi(cache: _Cache, q: np.ndarray, seq_lens, N: int, I: int, shard: int):
+    q = np.ascontiguousarray(q, dtype=np.float64)
+    sl = np.ascontiguousarray(seq_lens, dtype=np.int64)
+    B, QL, Hq, _ = q.shape
+    O = np.zeros((B, QL, Hq, cache.Dv), np.float64)
+    lse = np.zeros((B, QL, Hq), np.float64)
+    st = lib().orc_decode_multi(ctypes.byref(cache), _p(q), _p(sl), QL, N, I, shard, _p(O), _p(lse))
+    if st != ORC_OK:
+        raise ValueError(f"orc_decode_multi: bad arguments (status {st})")
+    return O, lse
+
+
+def decode_multi_arrays(kind: str, q, K, V, seq_lens, scale: float, dv: int | None = None,
+                        N: int = 1, I: int = 1, shard: int = -1):
+    """Decode with QL query tokens per request (speculative decoding under DCP, blog section 6):
+    q [B][QL][Hq][Dk]; request b holds seq_lens[b] positions, its QL new tokens last, and query
+    token j attends positions p <= seq_lens[b] - QL + j.  K, V, dv, N, I and shard as in
+    decode_arrays.  Returns O [B][QL][Hq][Dv], lse [B][QL][Hq]."""
+    q = np.asarray(q, np.float64)
+    B, QL, Hq, Dk = q.shape
+    K = np.ascontiguousarray(K, dtype=np.float64)
+    if kind == "mla":
+        Vd = dv if dv is not None else Dk
+        c = _Cache(1, 0, B, Hq, 1, Dk, Vd, scale, 0, _p(K).value, None, K.shape[1], 0)
+        keep = (K,)
+    else:
+        V = np.ascontiguousarray(V, dtype=np.float64)
+        c = _Cache(0, 0, B, Hq, K.shape[2], Dk, V.shape[3], scale, 0, _p(K).value, _p(V).value, K.shape[1], 0)
+        keep = (K, V)
+    out = _decode_multi(c, q, seq_lens, N, I, shard)
+    del keep
+    return out
 
 
 def merge(O_part: np.ndarray, lse_part: np.ndarray):

@@ -29,6 +29,10 @@
  *    a shard owning no position gives O = 0, LSE = -inf;
  *  - merge: M = max_n LSE_n, LSE = M + ln sum_n exp(LSE_n - M),
  *    O = sum_n exp(LSE_n - LSE) O_n;
+ *  - several query tokens per request (speculative decoding under DCP, blog
+ *    section 6): with L_b positions, the QL new ones last, query token j
+ *    attends the positions p <= L_b - QL + j (reading: the pages do not state
+ *    the mask; this is the causal one);
  *  - MLA (absorbed form): key = the whole 576-wide latent row, value = its
  *    first Dv entries;
  *  - fp8 latent cache (e4m3, OCP "E4M3" with no infinities, max 448) with a
@@ -238,18 +242,19 @@ static void fetch_row(const orc_cache* c, int32_t b, int64_t p, int32_t g, int i
         out[d] = bf16_to_double(synth_bf16_at(key, synth_kv_index(b, p, g, d, c->Hkv, W)));
 }
 
-/* One request b, the query heads h in [h0, h1) that all read kv head g.
- * Positions: all p < L, or (shard >= 0) only those owned by `shard`. */
-static void attend_group(const orc_cache* c, const double* q, int32_t b, int64_t L, int32_t g, int32_t h0,
-                         int32_t h1, int32_t N, int32_t I, int32_t shard, double* O, double* lse) {
+/* One query row set of request b (qb: [Hq][Dk]; results Ob: [Hq][Dv], lseb: [Hq]), the query heads
+ * h in [h0, h1) that all read kv head g.  Positions: all p < L, or (shard >= 0) only those owned
+ * by `shard`. */
+static void attend_group(const orc_cache* c, const double* qb, int32_t b, int64_t L, int32_t g, int32_t h0,
+                         int32_t h1, int32_t N, int32_t I, int32_t shard, double* Ob, double* lseb) {
     int32_t nh = h1 - h0, Dk = c->Dk, Dv = c->Dv;
     int64_t nsel = 0;
     if (shard < 0) nsel = L;
     else nsel = orc_shard_count(L, N, I, shard);
     if (nsel == 0) {
         for (int32_t h = h0; h < h1; h++) {
-            memset(O + ((int64_t)b * c->Hq + h) * Dv, 0, sizeof(double) * (size_t)Dv);
-            lse[(int64_t)b * c->Hq + h] = -INFINITY;
+            memset(Ob + (int64_t)h * Dv, 0, sizeof(double) * (size_t)Dv);
+            lseb[h] = -INFINITY;
         }
         return;
     }
@@ -267,7 +272,7 @@ static void attend_group(const orc_cache* c, const double* q, int32_t b, int64_t
         if (shard >= 0 && orc_owner(p, N, I) != shard) continue;
         fetch_row(c, b, p, g, 0, row, t16, t8);
         for (int32_t j = 0; j < nh; j++) {
-            const double* qh = q + ((int64_t)b * c->Hq + (h0 + j)) * Dk;
+            const double* qh = qb + (int64_t)(h0 + j) * Dk;
             double dot = 0.0;
             for (int32_t d = 0; d < Dk; d++) dot += qh[d] * row[d];
             double s = c->scale * dot;
@@ -279,7 +284,7 @@ static void attend_group(const orc_cache* c, const double* q, int32_t b, int64_t
     /* pass 2: l = sum exp(s - m), O = sum exp(s - m) v / l */
     for (int32_t j = 0; j < nh; j++) {
         l[j] = 0.0;
-        memset(O + ((int64_t)b * c->Hq + h0 + j) * Dv, 0, sizeof(double) * (size_t)Dv);
+        memset(Ob + (int64_t)(h0 + j) * Dv, 0, sizeof(double) * (size_t)Dv);
     }
     i = 0;
     for (int64_t p = 0; p < L; p++) {
@@ -288,15 +293,15 @@ static void attend_group(const orc_cache* c, const double* q, int32_t b, int64_t
         for (int32_t j = 0; j < nh; j++) {
             double w = exp(S[i * nh + j] - m[j]);
             l[j] += w;
-            double* Oh = O + ((int64_t)b * c->Hq + h0 + j) * Dv;
+            double* Oh = Ob + (int64_t)(h0 + j) * Dv;
             for (int32_t d = 0; d < Dv; d++) Oh[d] += w * row[d];
         }
         i++;
     }
     for (int32_t j = 0; j < nh; j++) {
-        double* Oh = O + ((int64_t)b * c->Hq + h0 + j) * Dv;
+        double* Oh = Ob + (int64_t)(h0 + j) * Dv;
         for (int32_t d = 0; d < Dv; d++) Oh[d] /= l[j];
-        lse[(int64_t)b * c->Hq + h0 + j] = m[j] + log(l[j]);
+        lseb[h0 + j] = m[j] + log(l[j]);
     }
     free(S); free(row); free(t16); free(t8); free(m); free(l);
 }
@@ -321,7 +326,39 @@ int orc_decode(const orc_cache* c, const double* q, const int64_t* seq_lens, int
         int32_t b = req_list ? req_list[r] : r;
         int32_t h0 = k * hb, h1 = h0 + hb > c->Hq ? c->Hq : h0 + hb;
         int32_t g = (c->kind == 1) ? 0 : h0 / group;
-        attend_group(c, q, b, seq_lens[b], g, h0, h1, N, I, shard, O, lse);
+        attend_group(c, q + (int64_t)b * c->Hq * c->Dk, b, seq_lens[b], g, h0, h1, N, I, shard,
+                     O + (int64_t)b * c->Hq * c->Dv, lse + (int64_t)b * c->Hq);
+    }
+    return ORC_OK;
+}
+
+/* Decode with QL query tokens per request (speculative decoding / multi-token prediction
+ * running under DCP: blog section 6).  Request b holds L_b positions, the QL new tokens
+ * included: query token j sits at position L_b - QL + j and attends the positions up to
+ * and including its own, p < L_b - QL + j + 1 (causal among the new tokens; reading: the
+ * pages name the combination but not the mask, and this is the standard one).
+ * q: [B][QL][Hq][Dk]; O: [B][QL][Hq][Dv]; lse: [B][QL][Hq].  Requires L_b >= QL.
+ * shard < 0: unsharded; shard = n: shard n's partial under (N, I). */
+int orc_decode_multi(const orc_cache* c, const double* q, const int64_t* seq_lens, int32_t QL, int32_t N,
+                     int32_t I, int32_t shard, double* O, double* lse) {
+    if (c->B < 1 || c->Hq < 1 || c->Hkv < 1 || c->Hq % c->Hkv || c->Dk < 1 || c->Dv < 1 || QL < 1) return ORC_ERR_ARG;
+    if (c->kind == 1 && (c->Hkv != 1 || c->Dv > c->Dk)) return ORC_ERR_ARG;
+    if (shard >= 0 && (N < 1 || I < 1 || shard >= N)) return ORC_ERR_ARG;
+    for (int32_t b = 0; b < c->B; b++)
+        if (seq_lens[b] < QL) return ORC_ERR_ARG;
+    int32_t group = c->Hq / c->Hkv;
+    int32_t hb = (c->kind == 1) ? (c->Hq < 16 ? c->Hq : 16) : group;
+    int32_t blocks = (c->Hq + hb - 1) / hb;
+    int64_t ntask = (int64_t)c->B * QL * blocks;
+#pragma omp parallel for schedule(dynamic, 1)
+    for (int64_t t = 0; t < ntask; t++) {
+        int64_t bj = t / blocks;
+        int32_t k = (int32_t)(t % blocks);
+        int32_t b = (int32_t)(bj / QL), j = (int32_t)(bj % QL);
+        int32_t h0 = k * hb, h1 = h0 + hb > c->Hq ? c->Hq : h0 + hb;
+        int32_t g = (c->kind == 1) ? 0 : h0 / group;
+        attend_group(c, q + bj * c->Hq * c->Dk, b, seq_lens[b] - QL + j + 1, g, h0, h1, N, I, shard,
+                     O + bj * c->Hq * c->Dv, lse + bj * c->Hq);
     }
     return ORC_OK;
 }

@@ -225,6 +225,102 @@ def test_mla_value_is_leading_slice_of_latent():
 
 
 # ----------------------------------------------------------------------------
+# several query tokens per request (speculative decoding under DCP, blog section 6)
+# ----------------------------------------------------------------------------
+
+def _brute_multi(q, K, V, L, scale, kind, dv=None):
+    """Masked softmax over ALL Lmax stored positions with the exponential taken directly:
+    query token j of request b may see position p iff p < L_b and p <= L_b - QL + j."""
+    B, QL, Hq, Dk = q.shape
+    Lmax = K.shape[1]
+    O = np.zeros((B, QL, Hq, dv if kind == "mla" else V.shape[3]))
+    lse = np.zeros((B, QL, Hq))
+    pos = np.arange(Lmax)
+    for b in range(B):
+        for j in range(QL):
+            visible = (pos < L[b]) & (pos <= L[b] - QL + j)
+            for h in range(Hq):
+                if kind == "mla":
+                    k, v = K[b], K[b, :, :dv]
+                else:
+                    g = h // (Hq // K.shape[2])
+                    k, v = K[b, :, g, :], V[b, :, g, :]
+                e = np.where(visible, np.exp(scale * (k @ q[b, j, h])), 0.0)
+                O[b, j, h] = (e[:, None] * v).sum(0) / e.sum()
+                lse[b, j, h] = math.log(e.sum())
+    return O, lse
+
+
+@pytest.mark.parametrize("QL", [1, 2, 4])
+def test_multi_query_brute_force_gqa(QL):
+    rng = np.random.default_rng(40 + QL)
+    B, Hq, Hkv, D, Lmax = 3, 4, 2, 8, 30
+    q = rng.standard_normal((B, QL, Hq, D))
+    K = rng.standard_normal((B, Lmax, Hkv, D))
+    V = rng.standard_normal((B, Lmax, Hkv, D + 2))
+    L = np.array([QL, 17, Lmax])  # the shortest request: its first query sees position 0 only
+    O, lse = oracle.decode_multi_arrays("gqa", q, K, V, L, 0.41)
+    Ob, lb = _brute_multi(q, K, V, L, 0.41, "gqa")
+    np.testing.assert_allclose(O, Ob, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, lb, rtol=1e-12, atol=1e-13)
+
+
+def test_multi_query_brute_force_mla():
+    rng = np.random.default_rng(7)
+    B, QL, Hq, Dk, Dv, Lmax = 2, 3, 16, 12, 8, 25
+    q = rng.standard_normal((B, QL, Hq, Dk))
+    K = rng.standard_normal((B, Lmax, Dk))
+    L = np.array([9, 25])
+    O, lse = oracle.decode_multi_arrays("mla", q, K, None, L, 0.3, dv=Dv)
+    Ob, lb = _brute_multi(q, K, None, L, 0.3, "mla", dv=Dv)
+    np.testing.assert_allclose(O, Ob, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lse, lb, rtol=1e-12, atol=1e-13)
+
+
+def test_multi_query_reduces_to_single_query_decode():
+    """QL = 1 is plain decode, and the last of QL query tokens sees the whole request."""
+    rng = np.random.default_rng(11)
+    B, Hq, Hkv, D, Lmax = 3, 6, 3, 5, 40
+    q, K, V = _rand_problem(rng, B, Hq, Hkv, D, D, Lmax)
+    L = np.array([4, 23, 40])
+    O1, l1 = oracle.decode_arrays("gqa", q, K, V, L, 0.5)
+    Om, lm = oracle.decode_multi_arrays("gqa", q[:, None], K, V, L, 0.5)
+    np.testing.assert_array_equal(Om[:, 0], O1)
+    np.testing.assert_array_equal(lm[:, 0], l1)
+    q4 = rng.standard_normal((B, 4, Hq, D))
+    O4, l4 = oracle.decode_multi_arrays("gqa", q4, K, V, L, 0.5)
+    Ol, ll = oracle.decode_arrays("gqa", q4[:, 3], K, V, L, 0.5)
+    np.testing.assert_array_equal(O4[:, 3], Ol)
+    np.testing.assert_array_equal(l4[:, 3], ll)
+
+
+@pytest.mark.parametrize("N,I", [(2, 1), (3, 2), (4, 5), (8, 1)])
+def test_multi_query_sharded_merge_reproduces_unsharded(N, I):
+    """The causal limit composes with the shard filter: per-shard partials of each query token
+    LSE-merge to its unsharded result."""
+    rng = np.random.default_rng(N * 7 + I)
+    B, QL, Hq, Hkv, D, Lmax = 2, 3, 4, 2, 6, 60
+    q = rng.standard_normal((B, QL, Hq, D))
+    K = rng.standard_normal((B, Lmax, Hkv, D))
+    V = rng.standard_normal((B, Lmax, Hkv, D))
+    L = np.array([3, 60])
+    O, lse = oracle.decode_multi_arrays("gqa", q, K, V, L, 0.3)
+    parts = [oracle.decode_multi_arrays("gqa", q, K, V, L, 0.3, N=N, I=I, shard=n) for n in range(N)]
+    Op = np.stack([p[0].reshape(B * QL, Hq, D) for p in parts])
+    Lp = np.stack([p[1].reshape(B * QL, Hq) for p in parts])
+    Om, lm = oracle.merge(Op, Lp)
+    np.testing.assert_allclose(Om.reshape(O.shape), O, rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(lm.reshape(lse.shape), lse, rtol=1e-12, atol=1e-13)
+
+
+def test_multi_query_rejects_requests_shorter_than_the_query():
+    q = np.zeros((1, 3, 2, 4))
+    K = np.zeros((1, 5, 1, 4))
+    with pytest.raises(ValueError):
+        oracle.decode_multi_arrays("gqa", q, K, K, [2], 1.0)
+
+
+# ----------------------------------------------------------------------------
 # sharding + merge invariant (pins the split into shards and chunks)
 # ----------------------------------------------------------------------------
 
