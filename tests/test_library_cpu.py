@@ -96,6 +96,64 @@ def test_host_validation_without_gpu():
     assert L.dcp_shard_map(ctypes.byref(d), 1, 16, None, 16, 16, 16, None) == dcp.DCP_ERR_MISALIGNED
 
 
+def _valid_mla_desc(dtype):
+    d = dcp.CacheDesc()
+    d.kind, d.dtype, d.n_shards, d.interleave, d.page_size = dcp.DCP_MLA, dtype, 2, 1, 64
+    d.num_pages, d.hq, d.hkv, d.dk, d.dv, d.batch, d.max_local_pages = 10, 64, 1, 576, 512, 1, 4
+    # placeholder addresses: the host checks read pointer values only, never the memory
+    d.k_pages, d.block_tables = 256, 16
+    d.kv_scales = 512 if dtype == dcp.DCP_FP8_E4M3 else None
+    return d
+
+
+def test_decode_host_validation_without_gpu():
+    """dcp_decode_partial and its no-alloc form reject bad descriptors and arguments with the status
+    include/dcp.h names, before any CUDA call."""
+    L = dcp.lib()
+    A = 1024  # a 16-byte-aligned placeholder device address
+
+    def part(d, B=1, q=A, seq=A, o=A, lse=A, ws=A):
+        return L.dcp_decode_partial(ctypes.byref(d), B, q, seq, o, lse, ws, 1 << 20, None)
+
+    def noalloc(d, B=1, q=A, seq=A, o=A, lse=A):
+        return L.dcp_decode_partial_noalloc(ctypes.byref(d), B, q, seq, o, lse, None)
+
+    for dt in (dcp.DCP_BF16, dcp.DCP_FP8_E4M3):
+        d = _valid_mla_desc(dt)
+        for f in (part, noalloc):
+            assert f(d, B=2) == dcp.DCP_ERR_INVALID_ARG          # B != cache->batch
+            assert f(d, q=None) == dcp.DCP_ERR_INVALID_ARG
+            assert f(d, lse=None) == dcp.DCP_ERR_INVALID_ARG
+            assert f(d, q=A + 8) == dcp.DCP_ERR_MISALIGNED
+            assert f(d, o=A + 4) == dcp.DCP_ERR_MISALIGNED
+        assert part(d, ws=None) == dcp.DCP_ERR_INVALID_ARG
+        assert part(d, ws=A + 8) == dcp.DCP_ERR_MISALIGNED
+    cases = [  # (field changes on a valid descriptor, expected status)
+        ({"hq": 8}, dcp.DCP_ERR_UNSUPPORTED),                  # MLA heads come in blocks of 16
+        ({"dk": 512}, dcp.DCP_ERR_UNSUPPORTED),
+        ({"dtype": 7}, dcp.DCP_ERR_INVALID_ARG),
+        ({"kind": 5}, dcp.DCP_ERR_INVALID_ARG),
+        ({"page_size": 32}, dcp.DCP_ERR_UNSUPPORTED),
+        ({"n_shards": 0}, dcp.DCP_ERR_INVALID_ARG),
+        ({"max_local_pages": 1 << 26}, dcp.DCP_ERR_INVALID_ARG),  # 2^26 pages x 64 tokens overflows int32
+        ({"k_pages": None}, dcp.DCP_ERR_INVALID_ARG),
+        ({"k_pages": 264}, dcp.DCP_ERR_MISALIGNED),
+        ({"block_tables": 20}, dcp.DCP_ERR_MISALIGNED),
+        ({"dtype": dcp.DCP_FP8_E4M3, "kv_scales": None}, dcp.DCP_ERR_INVALID_ARG),
+        ({"dtype": dcp.DCP_FP8_E4M3, "kv_scales": 520}, dcp.DCP_ERR_MISALIGNED),
+        ({"kind": dcp.DCP_GQA, "hkv": 4, "dk": 128, "dv": 64, "v_pages": 768}, dcp.DCP_ERR_UNSUPPORTED),
+        ({"kind": dcp.DCP_GQA, "hkv": 4, "dk": 128, "dv": 128, "v_pages": 768, "dtype": dcp.DCP_FP8_E4M3},
+         dcp.DCP_ERR_UNSUPPORTED),
+        ({"kind": dcp.DCP_GQA, "hkv": 4, "dk": 128, "dv": 128, "v_pages": None}, dcp.DCP_ERR_INVALID_ARG),
+    ]
+    for changes, want in cases:
+        d = _valid_mla_desc(dcp.DCP_BF16)
+        for k, v in changes.items():
+            setattr(d, k, v)
+        assert part(d) == want, changes
+        assert noalloc(d) == want, changes
+
+
 def test_libsynth_exports():
     lib = synth.device_lib()
     assert hasattr(lib, "synth_fill_flat") and hasattr(lib, "synth_fill_kv_rows")
