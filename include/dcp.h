@@ -221,8 +221,19 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
  *  the scratch; otherwise the planner's split-slot bound is shrunk (fewer
  *  units per CTA, so fewer, longer chunks) until it fits.  Returns
  *  DCP_ERR_WORKSPACE_TOO_SMALL, launching nothing, when even the smallest
- *  bound does not fit: the scratch grows with n_shards * B * hq (per-shard
- *  counters) and with hq * dv (split partials).
+ *  bound does not fit.  With T = u * C units targeted (u = units per CTA,
+ *  halved from 16 -- 4 for the CUDA-core paths -- down to 1; C = the persistent
+ *  grid: one CTA per SM for the tensor-core MLA path, SMs x resident CTAs per
+ *  SM for the others), the scratch holds, each term rounded up to 256 bytes:
+ *    32 * (N*B + T + 1)          work units
+ *    4 * N*B*hq + 8 * N*B        per-shard counters
+ *    4 * (2T + 2) * hq * (dv+1)  split-chunk partials and their LSE
+ *    B * (128*576 + 256)         fp8 MLA on tensor cores only: the query
+ *                                split into two e4m3 terms.
+ *  So the fp8 MLA path with B = 512 and hq = 64 (the high-concurrency
+ *  workload) does not fit at any N on a 148-SM part: its query split alone
+ *  takes 37.9 MB and the smallest split area 39 MB; such callers use
+ *  dcp_decode_partial with a workspace.
  *  The plan kernel, first on `stream`, clears the scratch's work ticket and
  *  done counters; nothing else in it needs initialising.
  *  Calls that can overlap in time (different streams, or threads without an

@@ -1,5 +1,7 @@
 // api.cu -- the C ABI of libdcp (include/dcp.h): host-side validation, the
 // sticky device status word, workspace sizing and kernel dispatch.
+#include <cudaTypedefs.h>
+
 #include <mutex>
 
 #include "common.cuh"
@@ -14,26 +16,84 @@ namespace {
 
 constexpr int kMaxDevices = 64;
 std::mutex g_mu;
-int* g_status_ptr[kMaxDevices] = {nullptr};
-int g_num_sms[kMaxDevices] = {0};
+
+// The addresses of this library's __device__ arrays belong to the CUDA context
+// that loaded the module: a context rebuilt after cudaDeviceReset reloads it
+// elsewhere.  So they are cached per device together with the id of the
+// context they were looked up in, and looked up again when that id changes.
+struct DeviceCache {
+    unsigned long long ctx_id = 0;
+    bool valid = false;
+    int* status = nullptr;
+    uint8_t* scratch = nullptr;  // built-in decode scratch, looked up on first use
+    int num_sms = 0;
+};
+DeviceCache g_dev[kMaxDevices];
+
+using PFN_ctxGetCurrent = CUresult (*)(CUcontext*);
+using PFN_ctxGetId = CUresult (*)(CUcontext, unsigned long long*);
+std::once_flag g_ctx_once;
+PFN_ctxGetCurrent g_ctx_get_current = nullptr;
+PFN_ctxGetId g_ctx_get_id = nullptr;
+
+void load_ctx_entries() {
+    void* fn = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_ctx_get_current = reinterpret_cast<PFN_ctxGetCurrent>(fn);
+    fn = nullptr;
+    if (cudaGetDriverEntryPoint("cuCtxGetId", &fn, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+        g_ctx_get_id = reinterpret_cast<PFN_ctxGetId>(fn);
+}
+
+// Id of the calling thread's current context (0 when none is current or the
+// driver cannot say).
+unsigned long long current_ctx_id() {
+    std::call_once(g_ctx_once, load_ctx_entries);
+    if (!g_ctx_get_current || !g_ctx_get_id) return 0;
+    CUcontext ctx = nullptr;
+    if (g_ctx_get_current(&ctx) != CUDA_SUCCESS || !ctx) return 0;
+    unsigned long long id = 0;
+    if (g_ctx_get_id(ctx, &id) != CUDA_SUCCESS) return 0;
+    return id;
+}
 
 dcp_status cuda_err(cudaError_t e) { return e == cudaSuccess ? DCP_OK : DCP_ERR_CUDA; }
 
-// device address of g_status and SM count of the current device
-dcp_status device_info(int** status, int* num_sms) {
+// The cache entry of the current device, valid for its current context.  Must
+// be called with g_mu held.
+dcp_status device_entry(DeviceCache** out) {
     int dev = 0;
     if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DCP_ERR_CUDA;
-    std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_status_ptr[dev]) {
+    DeviceCache& d = g_dev[dev];
+    unsigned long long id = current_ctx_id();
+    if (!d.valid || id == 0 || id != d.ctx_id) {
+        // cudaGetSymbolAddress makes the device's primary context current when
+        // none is, so the id is read again after it
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_status) != cudaSuccess) return DCP_ERR_CUDA;
         int sms = 0;
         if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return DCP_ERR_CUDA;
-        g_status_ptr[dev] = static_cast<int*>(p);
-        g_num_sms[dev] = sms;
+        d.status = static_cast<int*>(p);
+        d.scratch = nullptr;
+        d.num_sms = sms;
+        d.ctx_id = current_ctx_id();
+        d.valid = true;
     }
-    if (status) *status = g_status_ptr[dev];
-    if (num_sms) *num_sms = g_num_sms[dev];
+    *out = &d;
+    return DCP_OK;
+}
+
+// device address of g_status and SM count of the current device
+dcp_status device_info(int** status, int* num_sms) {
+    std::lock_guard<std::mutex> lk(g_mu);
+    DeviceCache* d = nullptr;
+    dcp_status st = device_entry(&d);
+    if (st != DCP_OK) return st;
+    if (status) *status = d->status;
+    if (num_sms) *num_sms = d->num_sms;
     return DCP_OK;
 }
 
@@ -98,21 +158,21 @@ bool make_plan(const dcp_cache_desc* c, int B, int num_sms, Plan* p) {
 // ---------------------------------------------------------------------------
 // built-in decode scratch (dcp_decode_partial_noalloc)
 // ---------------------------------------------------------------------------
-// One per device context; its address is looked up once per device.
+// One per device context.  Its address is looked up on the first no-alloc call
+// in a context (and again if the context is rebuilt), with that device current.
 static __device__ __align__(256) uint8_t g_decode_scratch[DCP_STATIC_SCRATCH_BYTES];
 
-uint8_t* g_scratch_ptr[kMaxDevices] = {nullptr};
-
 dcp_status decode_scratch(uint8_t** out) {
-    int dev = 0;
-    if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return DCP_ERR_CUDA;
     std::lock_guard<std::mutex> lk(g_mu);
-    if (!g_scratch_ptr[dev]) {
+    DeviceCache* d = nullptr;
+    dcp_status st = device_entry(&d);
+    if (st != DCP_OK) return st;
+    if (!d->scratch) {
         void* p = nullptr;
         if (cudaGetSymbolAddress(&p, g_decode_scratch) != cudaSuccess) return DCP_ERR_CUDA;
-        g_scratch_ptr[dev] = static_cast<uint8_t*>(p);
+        d->scratch = static_cast<uint8_t*>(p);
     }
-    *out = g_scratch_ptr[dev];
+    *out = d->scratch;
     return DCP_OK;
 }
 

@@ -25,10 +25,13 @@
 // maximum is rescaled lazily: O^T is rescaled only when a head's maximum grows
 // by more than 2^8 (P then stays below 256).
 //
-// Warp roles (one CTA per SM, persistent, units taken from an atomic ticket):
+// Warp roles (224 threads, one CTA per SM, persistent, units taken from an
+// atomic ticket):
 //   warp 0      TMA producer (lane 0): nine [64][64] boxes per tile, 128 B swizzle
-//   warp 1      TMEM allocation, MMA issue (lane 0)
-//   warps 2..5  softmax, lazy rescale of O^T, epilogue (one per TMEM lane quadrant)
+//   warp 1      TMEM allocation; lane 0 issues the S MMAs of each tile
+//   warps 2..5  softmax, lazy rescale of O^T, epilogue (one per TMEM lane
+//               quadrant; lanes l and l + 16 share head l's 64 tokens)
+//   warp 6      lane 0 issues the P V MMAs of each tile
 #include "common.cuh"
 #include "finish.cuh"
 #include "kernels.h"
