@@ -4,8 +4,8 @@
 One step = one pass of the whole hot path over the batch, for one new token
 per request:
   dcp_shard_map (owner/slot of position L_b)  ->  dcp_kv_append (write the new
-  token into its owner's page)  ->  dcp_decode_partial (all N shards' partial
-  attention over positions [0, L_b + 1))  ->  dcp_merge (LSE merge).
+  token into its owner's page)  ->  dcp_decode_merged (every shard's partial
+  attention over positions [0, L_b + 1) and the LSE merge, fused).
 Lengths grow by one token per step, as in decoding.
 
 Metric: KV GB/s = (sum_b attended tokens x KV bytes per token) / step time,
@@ -13,6 +13,19 @@ plus decode steps/s, and the fraction of the measured HBM copy bandwidth.
 Inputs are synthetic (seeded generator) with the shapes of the named
 workload; the KV cache (>= several GB) is far larger than the 126 MB L2, so
 no L2 flush is needed between steps.
+
+The JSON line's headline is one workload (--config, default the
+high-concurrency fp8 MLA one); at N = 1 the two other large workloads (GQA
+Qwen3-shaped, MLA Kimi-shaped bf16) are measured the same way under
+"per_config".  Each workload also reports:
+  - "bands": per-request completion time inside the full batch, by request
+    length band (<32k, 32-64k, 64-128k, 128-200k, 200k+), from the device
+    timestamps dcp_decode_merged records per request;
+  - "fused_vs_unfused": dcp_decode_merged against dcp_decode_partial +
+    dcp_merge on the same inputs;
+  - "e2e": the same step through the C ABI with host buffers, the inputs copied
+    in and the output copied out every step on copy streams overlapped with
+    the previous / next step's compute.
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--config 5]
                   [--n-shards 8] [--interleave 1] [--impl ours|reference]
@@ -53,13 +66,14 @@ def parse():
     ap.add_argument("--warmup", type=int, default=5)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--config", type=int, default=HEADLINE_CONFIG)
+    ap.add_argument("--per-config", default="3,4",
+                    help="other workloads measured the same way at N = 1 ('' for none)")
     ap.add_argument("--n-shards", type=int, default=None)
     ap.add_argument("--interleave", type=int, default=None)
     ap.add_argument("--batch-limit", type=int, default=None,
                     help="keep only the first B requests of the workload (small profiling cases)")
     ap.add_argument("--no-e2e", action="store_true")
-    ap.add_argument("--bands", action="store_true",
-                    help="also time the decode per request-length band (<32k, 32-64k, 64-128k, 128-200k, 200k+)")
+    ap.add_argument("--no-bands", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=25.0, help="target CPU work of the oracle sample")
     return ap.parse_args()
@@ -73,16 +87,18 @@ def peaks():
     return 6650.0, "fallback"
 
 
-def get_workload(args):
-    w = synth.workload(args.config, n_shards=args.n_shards, interleave=args.interleave)
-    if args.batch_limit:
+def get_workload(args, cfg=None):
+    cfg = args.config if cfg is None else cfg
+    own = cfg == args.config
+    w = synth.workload(cfg, n_shards=args.n_shards if own else None, interleave=args.interleave if own else None)
+    if args.batch_limit and own:
         w.B = min(w.B, args.batch_limit)
         w.lengths = w.lengths[:w.B]
     return w
 
 
-def workload_config(w, args):
-    return {"workload": f"config{args.config}: {w.name}", "kind": w.kind, "kv_dtype": w.dtype,
+def workload_config(w, cfg):
+    return {"workload": f"config{cfg}: {w.name}", "kind": w.kind, "kv_dtype": w.dtype,
             "batch": w.B, "q_heads": w.hq, "kv_heads": w.hkv, "dk": w.dk, "dv": w.dv, "page_size": w.page_size,
             "n_shards": w.n_shards, "interleave": w.interleave, "total_tokens": int(np.sum(w.lengths)),
             "median_len": int(np.median(w.lengths)), "max_len": int(np.max(w.lengths)),
@@ -196,25 +212,24 @@ def measured_traffic(config_key: str):
     return float(e["dram_bytes_per_launch"])
 
 
-def traffic_key(args, w) -> str:
-    return f"config{args.config} B{w.B} N{w.n_shards} I{w.interleave}"
+def traffic_key(cfg, w) -> str:
+    return f"config{cfg} B{w.B} N{w.n_shards} I{w.interleave}"
 
 
 def launches_per_step(w) -> int:
-    """Kernels one step launches: shard map, append, plan, [query split], decode, merge."""
+    """Kernels one step launches: shard map, append, plan, [query split], decode (merged)."""
     fp8_tc = w.kind == "mla" and w.dtype == "fp8" and w.hq in (16, 32, 64) and w.page_size == 64
-    return 6 if fp8_tc else 5
+    return 5 if fp8_tc else 4
 
 
-def combine_ranks(dist, device, ms, kern_total, e2e_ms, bytes_timed, e2e_bytes):
-    """Max over ranks of the device times, sum over ranks of the bytes."""
+def combine_ranks(dist, device, times, sums):
+    """Max over ranks of the device times, sum over ranks of the byte counts."""
     import torch
-    t = torch.tensor([ms, kern_total, e2e_ms], dtype=torch.float64, device=device)
+    t = torch.tensor([float(x) for x in times], dtype=torch.float64, device=device)
     dist.all_reduce(t, op=dist.ReduceOp.MAX)
-    tb = torch.tensor([float(bytes_timed), float(e2e_bytes)], dtype=torch.float64, device=device)
+    tb = torch.tensor([float(x) for x in sums], dtype=torch.float64, device=device)
     dist.all_reduce(tb, op=dist.ReduceOp.SUM)
-    (ms, kern_total, e2e_ms), (b, eb) = t.tolist(), tb.tolist()
-    return ms, kern_total, e2e_ms, b, eb
+    return t.tolist(), tb.tolist()
 
 
 # ----------------------------------------------------------------------------
@@ -225,33 +240,30 @@ BANDS = [(0, 32_000, "<32k"), (32_000, 64_000, "32-64k"), (64_000, 128_000, "64-
          (128_000, 200_000, "128-200k"), (200_000, 1 << 31, "200k+")]
 
 
-def time_bands(args, w, dcp, dw, q, lens, o_part, lse, stream, reps: int = 5):
-    """Decode time per request-length band: the other requests get length 0 (their
-    shards are empty), so the launch covers exactly the band's tokens."""
-    import torch
+def band_latency(lengths, finish_ms, decode_ms, kv_bytes_per_token):
+    """Per-request completion times inside one full-batch decode, by length band.
+    finish_ms[b]: request b's output stored, ms after the decode's first kernel
+    started (median over repeated launches)."""
+    L = np.asarray(lengths)
     out = {}
-    L = lens.cpu().numpy()
     for lo, hi, name in BANDS:
         sel = (L >= lo) & (L < hi)
         if not sel.any():
             continue
-        lb = torch.as_tensor(np.where(sel, L, 0).astype(np.int32), device=lens.device)
-        for _ in range(2):
-            dcp.dcp_decode_partial(dw.desc, q, lb, o_part, lse, dw.ws)
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            dcp.dcp_decode_partial(dw.desc, q, lb, o_part, lse, dw.ws)
-        e1.record(stream)
-        torch.cuda.synchronize()
-        ms = e0.elapsed_time(e1) / reps
+        f = np.asarray(finish_ms)[sel]
         tok = int(L[sel].sum())
-        out[name] = {"requests": int(sel.sum()), "tokens": tok, "decode_ms": round(ms, 4),
-                     "kv_gbs": round(tok * w.kv_bytes_per_token / (ms * 1e-3) / 1e9, 1)}
+        out[name] = {"requests": int(sel.sum()), "tokens": tok,
+                     "done_ms_p50": round(float(np.percentile(f, 50)), 4),
+                     "done_ms_p99": round(float(np.percentile(f, 99)), 4),
+                     "done_ms_max": round(float(f.max()), 4),
+                     "kv_gbs_by_band_done": round(tok * kv_bytes_per_token / (float(f.max()) * 1e-3) / 1e9, 1)}
+    out["batch_decode_ms"] = round(decode_ms, 4)
     return out
 
 
-def run_ours(args, rank, world, local_rank):
+def measure(args, cfg, rank, world, local_rank, headline):
+    """Time the decode step of workload `cfg` (see the module docstring); returns the
+    result dict (value, ms_per_step, roofline, clocks, e2e, bands, ...) and the workload."""
     import torch
     import torch.distributed as dist
 
@@ -260,20 +272,20 @@ def run_ours(args, rank, world, local_rank):
     from sequence_sharded_paged_b200 import workload as wl
 
     dcp.lib()  # fail loudly if libdcp.so is missing
-    torch.cuda.set_device(local_rank)
     dev = torch.device("cuda", local_rank)
-    w = get_workload(args)
+    w = get_workload(args, cfg)
     w.seed_val += 100 * rank  # each rank decodes its own independent batch
     E = 0 if args.no_e2e else args.steps
-    growth = args.warmup + args.steps + E + 1
+    n_total = args.warmup + args.steps + E
+    growth = n_total + 1
     counts = wl.gpu_shard_counts(np.asarray(w.lengths) + growth, w.n_shards, w.interleave)
     t0 = time.time()
     dw = wl.build(w, counts)
     fill_s = time.time() - t0
     B, N = w.B, w.n_shards
     L0 = torch.as_tensor(np.asarray(w.lengths, np.int32), device=dev)
+    ws = torch.empty(dcp.dcp_decode_workspace_size_ex(dw.desc, B, 1, True), dtype=torch.uint8, device=dev)
 
-    n_total = args.warmup + args.steps + E
     # per-step inputs, resident in HBM before the timed region
     qs = [sdev.q(w.seed_val, B, w.hq, w.dk, step=s + 1) for s in range(n_total)]
     req = torch.arange(B, dtype=torch.int32, device=dev)
@@ -286,22 +298,21 @@ def run_ours(args, rank, world, local_rank):
     rank_o = torch.empty(B, dtype=torch.int32, device=dev)
     local_o = torch.empty(B, dtype=torch.int32, device=dev)
     slot_o = torch.empty(B, dtype=torch.int64, device=dev)
-    o_part = torch.empty((N, B, w.hq, w.dv), dtype=torch.float32, device=dev)
-    lse = torch.empty((N, B, w.hq), dtype=torch.float32, device=dev)
     out = torch.empty((B, w.hq, w.dv), dtype=torch.float32, device=dev)
     lse_out = torch.empty((B, w.hq), dtype=torch.float32, device=dev)
     stream = torch.cuda.current_stream()
 
-    def step(s, ev=None):
-        dcp.dcp_shard_map(dw.desc, pos_s[s], None, rank_o, local_o, slot_o)
-        k, v = new_rows[s]
-        dcp.dcp_kv_append(dw.desc, None, pos_s[s], k, v)
+    def step(s, ev=None, pos=None, lens=None, q=None, k=None, v=None, o=out, lo=lse_out):
+        pos = pos_s[s] if pos is None else pos
+        if k is None:
+            k, v = new_rows[s]
+        dcp.dcp_shard_map(dw.desc, pos, None, rank_o, local_o, slot_o)
+        dcp.dcp_kv_append(dw.desc, None, pos, k, v)
         if ev is not None:
-            ev[0].record(stream)
-        dcp.dcp_decode_partial(dw.desc, qs[s], lens_s[s], o_part, lse, dw.ws)
+            ev[0].record(torch.cuda.current_stream())
+        dcp.dcp_decode_merged(dw.desc, qs[s] if q is None else q, lens_s[s] if lens is None else lens, o, lo, ws)
         if ev is not None:
-            ev[1].record(stream)
-        dcp.dcp_merge(o_part, lse, out, lse_out)
+            ev[1].record(torch.cuda.current_stream())
 
     clocks = Clocks(local_rank)
     clocks.start()
@@ -338,94 +349,135 @@ def run_ours(args, rank, world, local_rank):
     kern_ms = [a.elapsed_time(b) for a, b in ev_k]
     bytes_timed = sum(kv_tok[args.warmup + i] for i in range(args.steps)) * bpt
 
-    bands = time_bands(args, w, dcp, dw, qs[args.warmup], lens_s[args.warmup], o_part, lse, stream) \
-        if args.bands else None
+    # extra launches on the last timed step's inputs (untimed in `value`): per-request
+    # completion times, and the fused call against partial + merge
+    last = args.warmup + args.steps - 1
+    reps = 5
+    bands = None
+    if not args.no_bands:
+        fin = torch.zeros((reps, B), dtype=torch.int64, device=dev)
+        for r in range(reps):
+            dcp.dcp_decode_merged(dw.desc, qs[last], lens_s[last], out, lse_out, ws, finish_ns=fin[r])
+        torch.cuda.synchronize()
+        finish_ms = np.median(fin.cpu().numpy(), axis=0) / 1e6
+        bands = band_latency(np.asarray(w.lengths) + last + 1, finish_ms, float(np.median(kern_ms)), bpt)
+    ws_p = torch.empty(dcp.dcp_decode_workspace_size(dw.desc, B), dtype=torch.uint8, device=dev)
+    o_part = torch.empty((N, B, w.hq, w.dv), dtype=torch.float32, device=dev)
+    lse_p = torch.empty((N, B, w.hq), dtype=torch.float32, device=dev)
+    fu = {}
+    for name, fn in (("merged", lambda: dcp.dcp_decode_merged(dw.desc, qs[last], lens_s[last], out, lse_out, ws)),
+                     ("partial_plus_merge", lambda: (dcp.dcp_decode_partial(dw.desc, qs[last], lens_s[last], o_part,
+                                                                            lse_p, ws_p),
+                                                     dcp.dcp_merge(o_part, lse_p, out, lse_out)))):
+        fn()
+        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        e0.record(stream)
+        for _ in range(reps):
+            fn()
+        e1.record(stream)
+        torch.cuda.synchronize()
+        fu[name + "_ms"] = round(e0.elapsed_time(e1) / reps, 4)
+    del o_part, lse_p, ws_p
 
-    # end to end through the C ABI with host buffers: H2D of the step's inputs
-    # (q, new token rows, positions, lengths) from pinned memory, D2H of out + lse
+    # end to end through the C ABI with host buffers: each step's inputs (q, new token
+    # rows, positions, lengths) are copied in from pinned memory on one copy stream and
+    # its output (out + lse) copied back on another, double-buffered so that the copies
+    # of steps s - 1 and s + 1 overlap the compute of step s
     e2e = None
     if E:
+        first_e = args.warmup + args.steps
         pin = []
-        for s in range(args.warmup + args.steps, n_total):
+        for s in range(first_e, n_total):
             k, v = new_rows[s]
             pin.append((qs[s].cpu().pin_memory(), k.cpu().pin_memory(), None if v is None else v.cpu().pin_memory(),
                         pos_s[s].cpu().pin_memory(), lens_s[s].cpu().pin_memory()))
-        q_d, k_d = torch.empty_like(qs[0]), torch.empty_like(new_rows[0][0])
-        v_d = None if new_rows[0][1] is None else torch.empty_like(new_rows[0][1])
-        pos_d, len_d = torch.empty_like(pos_s[0]), torch.empty_like(lens_s[0])
-        out_h = torch.empty(out.shape, dtype=out.dtype).pin_memory()
-        lse_h = torch.empty(lse_out.shape, dtype=lse_out.dtype).pin_memory()
+        bufs = [tuple(None if t is None else torch.empty(t.shape, dtype=t.dtype, device=dev) for t in pin[0])
+                for _ in range(2)]
+        outs = [(torch.empty_like(out), torch.empty_like(lse_out)) for _ in range(2)]
+        host_out = [(torch.empty(out.shape, dtype=out.dtype).pin_memory(),
+                     torch.empty(lse_out.shape, dtype=lse_out.dtype).pin_memory()) for _ in range(2)]
         h2d = sum(t.numel() * t.element_size() for t in pin[0] if t is not None)
-        d2h = out_h.numel() * 4 + lse_h.numel() * 4
+        d2h = out.numel() * 4 + lse_out.numel() * 4
+        s_in, s_out = torch.cuda.Stream(device=dev), torch.cuda.Stream(device=dev)
+        ev_in = [torch.cuda.Event() for _ in range(2)]
+        ev_done = [torch.cuda.Event() for _ in range(2)]
+        ev_out = [torch.cuda.Event() for _ in range(2)]
         e0 = torch.cuda.Event(enable_timing=True)
         e1 = torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         e0.record(stream)
-        for i, (qh, kh, vh, ph, lh) in enumerate(pin):
-            q_d.copy_(qh, non_blocking=True)
-            k_d.copy_(kh, non_blocking=True)
-            if vh is not None:
-                v_d.copy_(vh, non_blocking=True)
-            pos_d.copy_(ph, non_blocking=True)
-            len_d.copy_(lh, non_blocking=True)
-            dcp.dcp_shard_map(dw.desc, pos_d, None, rank_o, local_o, slot_o)
-            dcp.dcp_kv_append(dw.desc, None, pos_d, k_d, v_d)
-            dcp.dcp_decode_partial(dw.desc, q_d, len_d, o_part, lse, dw.ws)
-            dcp.dcp_merge(o_part, lse, out, lse_out)
-            out_h.copy_(out, non_blocking=True)
-            lse_h.copy_(lse_out, non_blocking=True)
+        s_in.wait_event(e0)
+        s_out.wait_event(e0)
+        for i, host in enumerate(pin):
+            j = i % 2
+            with torch.cuda.stream(s_in):
+                if i >= 2:
+                    s_in.wait_event(ev_done[j])  # step i - 2 has consumed this input buffer
+                for dst, src in zip(bufs[j], host):
+                    if src is not None:
+                        dst.copy_(src, non_blocking=True)
+                ev_in[j].record(s_in)
+            stream.wait_event(ev_in[j])
+            if i >= 2:
+                stream.wait_event(ev_out[j])  # step i - 2's output has been copied out
+            q_d, k_d, v_d, p_d, l_d = bufs[j]
+            step(first_e + i, pos=p_d, lens=l_d, q=q_d, k=k_d, v=v_d, o=outs[j][0], lo=outs[j][1])
+            ev_done[j].record(stream)
+            with torch.cuda.stream(s_out):
+                s_out.wait_event(ev_done[j])
+                host_out[j][0].copy_(outs[j][0], non_blocking=True)
+                host_out[j][1].copy_(outs[j][1], non_blocking=True)
+                ev_out[j].record(s_out)
+        stream.wait_stream(s_out)
         e1.record(stream)
         torch.cuda.synchronize()
         if world > 1:
             dist.barrier()
+        st = dcp.dcp_get_device_status()
+        if st != dcp.DCP_OK:
+            raise RuntimeError(f"device status after the end-to-end steps: {dcp.status_string(st)}")
         e2e_ms = e0.elapsed_time(e1)
-        e2e_bytes = sum(kv_tok[args.warmup + args.steps + i] for i in range(E)) * bpt
+        e2e_bytes = sum(kv_tok[first_e + i] for i in range(E)) * bpt
         e2e = (e2e_ms, e2e_bytes, h2d, d2h)
 
     # max over ranks of device time; whole-job bytes
+    kern_total = sum(kern_ms)
     if world > 1:
-        ms, kern_total, e2e_ms_max, bytes_all, e2e_bytes_all = combine_ranks(
-            dist, dev, ms, sum(kern_ms), e2e[0] if e2e else 0.0, bytes_timed, e2e[1] if e2e else 0)
+        (ms, kern_total, e2e_ms_max), (bytes_all, e2e_bytes_all) = combine_ranks(
+            dist, dev, [ms, kern_total, e2e[0] if e2e else 0.0], [bytes_timed, e2e[1] if e2e else 0])
     else:
-        kern_total = sum(kern_ms)
         bytes_all = float(bytes_timed)
         e2e_ms_max = e2e[0] if e2e else 0.0
         e2e_bytes_all = float(e2e[1]) if e2e else 0.0
 
     hbm, peak_kind = peaks()
-    traffic = measured_traffic(traffic_key(args, w))
+    traffic = measured_traffic(traffic_key(cfg, w))
     gbs = bytes_all / (ms * 1e-3) / 1e9
-    # dominant kernel: the decode (plan + split-KV attention) of one step, CUDA events on its stream
+    # dominant kernel: the decode (plan + split-KV attention + merge) of one step, CUDA
+    # events on its stream
     per_launch_bytes = bytes_timed / args.steps
     kern_avg_ms = kern_total / args.steps
     achieved = per_launch_bytes / (kern_avg_ms * 1e-3) / 1e9
     res = {
-        "metric": METRIC,
         "value": round(gbs, 1),
         "unit": "GB/s",
-        "n_gpus": world,
-        "steps": args.steps,
-        "warmup": args.warmup,
         "ms_per_step": round(ms / args.steps, 4),
         "steps_per_s": round(args.steps / (ms * 1e-3), 2),
         "pct_hbm_measured": round(100 * gbs / world / hbm, 1),
         "pct_hbm_nominal_8tbs": round(100 * gbs / world / 8000.0, 1),
-        "higher_is_better": True,
-        "scaling": "weak",
-        "vs_baseline": None,
         "dtype": "bf16" if w.dtype == "bf16" else "fp8_e4m3 cache, bf16 q, fp32 accumulate",
-        "data": "synthetic (seeded counter-based generator; lengths shaped like the agentic trace)",
-        "config": workload_config(w, args) | {"parallelism": f"replicas x{world} (one independent batch per GPU)"},
+        "config": workload_config(w, cfg) | {"parallelism": f"replicas x{world} (one independent batch per GPU)"},
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 3), "traffic": traffic,
                      "algorithmic_bytes_per_launch": int(per_launch_bytes),
-                     "kernel": "dcp_decode_partial (planner + split-KV attention)",
+                     "kernel": "dcp_decode_merged (planner + split-KV attention + in-kernel LSE merge)",
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
-                     else "fallback 6650 GB/s"},
+                     else "fallback 6650 GB/s (no MEASURED_PEAKS.json)"},
         "clocks": clk,
         "gpu_launches": launches_per_step(w) * args.steps,
+        "fused_vs_unfused": fu,
         "fill_seconds": round(fill_s, 2),
     }
     if bands is not None:
@@ -433,7 +485,10 @@ def run_ours(args, rank, world, local_rank):
     if e2e:
         res["e2e"] = {"value": round(e2e_bytes_all / (e2e_ms_max * 1e-3) / 1e9, 1), "unit": "GB/s",
                       "h2d_bytes_per_step": e2e[2], "d2h_bytes_per_step": e2e[3],
-                      "ms_per_step": round(e2e_ms_max / E, 4)}
+                      "ms_per_step": round(e2e_ms_max / E, 4),
+                      "copies": "H2D and D2H on two copy streams, double-buffered, overlapping compute"}
+    del dw, ws, qs, new_rows
+    torch.cuda.empty_cache()
     return res, w
 
 
@@ -506,7 +561,7 @@ def run_reference(args):
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(dt / args.steps * 1e3, 2),
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
         "data": "synthetic (seeded counter-based generator)",
-        "config": workload_config(w, args) | {"parallelism": "host cores (OpenMP)"},
+        "config": workload_config(w, args.config) | {"parallelism": "host cores (OpenMP)"},
         "cpu_baseline": {"value": round(gbs, 4), "unit": "GB/s", "cores": oracle.num_threads(), "kind": "oracle",
                          "sample": sample},
         "e2e": {"value": round(gbs, 4), "unit": "GB/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
@@ -524,13 +579,27 @@ def main():
         return
     import torch
     import torch.distributed as dist
+    torch.cuda.set_device(local_rank)
     if world > 1:
         import datetime
-        torch.cuda.set_device(local_rank)
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        res, w = run_ours(args, rank, world, local_rank)
+        r, w = measure(args, args.config, rank, world, local_rank, True)
+        res = {"metric": METRIC, "value": r["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
+               "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "steps_per_s": r["steps_per_s"],
+               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": r["dtype"],
+               "data": "synthetic (seeded counter-based generator; lengths shaped like the agentic trace)"}
+        res.update({k: v for k, v in r.items() if k not in res})
+        others = [int(c) for c in args.per_config.split(",") if c.strip()] if world == 1 else []
+        per = {}
+        for cfg in others:
+            if cfg == args.config:
+                continue
+            rc, _ = measure(args, cfg, rank, world, local_rank, False)
+            per[f"config{cfg}"] = rc
+        if per:
+            res["per_config"] = per
         if rank == 0 and not args.no_cpu_baseline:
             cb, _, _ = time_oracle(w, args.cpu_seconds)
             res["cpu_baseline"] = cb

@@ -200,6 +200,71 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
                               float* o_partial, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * dcp_decode_workspace_size_ex -- bytes of device workspace that
+ * dcp_decode_partial_multi (merged = 0) or dcp_decode_merged (merged != 0)
+ * needs for this cache, batch and query length on the CURRENT device (host
+ * function; no GPU work).  Returns 0 for an invalid descriptor or a shape no
+ * kernel of this build covers.
+ */
+size_t dcp_decode_workspace_size_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_len, int32_t merged);
+
+/*
+ * dcp_decode_partial_multi -- dcp_decode_partial with q_len query tokens per
+ * request: speculative decoding / multi-token prediction under DCP.
+ * Passage: blog section 6 (future work: support for MTP and speculative
+ * decoding with DCP) on top of section 4.1.  The pages do not state the mask;
+ * this library takes the causal one: request b's last q_len positions are its
+ * new tokens, and query token j attends the positions p <= L_b - q_len + j.
+ *  q_len      1 <= q_len <= 64.  q_len > 1 is served by the tensor-core
+ *             kernels only: MLA with 64-token pages and q_len * hq in
+ *             {16, 32, 64}; GQA with q_len * hq / hkv == 16.  Other shapes
+ *             return DCP_ERR_UNSUPPORTED.
+ *  q          bf16 [B][q_len][hq][dk].
+ *  seq_lens   int32 [B]: L_b, which must be 0 or >= q_len (0 < L_b < q_len
+ *             records DCP_ERR_INVALID_ARG in the device status word; such a
+ *             request's token j attends max(0, L_b - q_len + j + 1) positions).
+ *  o_partial  fp32 [N][B][q_len][hq][dv]: shard n's normalised partial of each
+ *             query token over the positions it owns and that token attends;
+ *             0 where there are none.
+ *  lse        fp32 [N][B][q_len][hq]: natural-log LSE, -inf where none.
+ *  ws, ws_bytes  workspace of at least dcp_decode_workspace_size_ex(cache, B,
+ *             q_len, 0) bytes; clobbered.
+ * Errors as dcp_decode_partial.
+ */
+dcp_status dcp_decode_partial_multi(const dcp_cache_desc* cache, int32_t B, int32_t q_len, const void* q,
+                                    const int32_t* seq_lens, float* o_partial, float* lse, void* ws, size_t ws_bytes,
+                                    void* stream);
+
+/*
+ * dcp_decode_merged -- every shard's partial attention AND the LSE merge in
+ * one launch sequence: the output of dcp_decode_partial(_multi) followed by
+ * dcp_merge, without the per-shard partials ever being written as a whole.
+ * Passage: blog section 4.1 (each GPU's partial output and LSE, reweighted by
+ * the LSE values and summed by the all-gather + reduce-scatter).  Here all
+ * shards are on one GPU: the chunks of every shard of a request form one merge
+ * group, run side by side, and the last of them to finish merges the group's
+ * partials while they are still in L2 (then drops them from L2).
+ *  q_len, q, seq_lens   as dcp_decode_partial_multi (q_len = 1: one query
+ *             token per request, q bf16 [B][hq][dk]).
+ *  out        fp32 [B][q_len][hq][dv]: sum over shards of exp(lse_n - LSE) o_n,
+ *             i.e. the unsharded decode attention; 0 where a query token
+ *             attends no position.
+ *  lse_out    fp32 [B][q_len][hq]: LSE = M + ln sum_n exp(lse_n - M),
+ *             M = max_n lse_n; -inf where a query token attends no position.
+ *  finish_ns  int64 [B] or NULL: nanoseconds (device global timer) from the
+ *             start of the call's first kernel until request b's output was
+ *             stored.  For per-request latency within one batch; the values
+ *             order the requests' completions, they are not a kernel timer.
+ *  ws, ws_bytes  workspace of at least dcp_decode_workspace_size_ex(cache, B,
+ *             q_len, 1) bytes; clobbered.  Concurrent calls need distinct
+ *             workspaces.
+ * Errors as dcp_decode_partial (finish_ns must be 16-byte aligned too).
+ */
+dcp_status dcp_decode_merged(const dcp_cache_desc* cache, int32_t B, int32_t q_len, const void* q,
+                             const int32_t* seq_lens, float* out, float* lse_out, int64_t* finish_ns, void* ws,
+                             size_t ws_bytes, void* stream);
+
+/*
  * DCP_STATIC_SCRATCH_BYTES -- size of the decode scratch built into the
  * library: 64 MiB of device memory per device, reserved when the library's
  * device code is loaded on that device.

@@ -270,6 +270,19 @@ def decode_multi_arrays(kind: str, q, K, V, seq_lens, scale: float, dv: int | No
     return out
 
 
+def decode_multi_synth(kind: str, dtype: str, seed: int, q, seq_lens, scale: float, hkv: int, dk: int, dv: int,
+                       N: int = 1, I: int = 1, shard: int = -1):
+    """decode_multi_arrays with K/V (or latent) rows regenerated on the fly from the
+    seeded generator, as decode_synth does: q [B][QL][Hq][Dk] -> O [B][QL][Hq][Dv],
+    lse [B][QL][Hq]."""
+    q = np.asarray(q, np.float64)
+    B, QL, Hq, Dk = q.shape
+    assert Dk == dk
+    c = _Cache(1 if kind == "mla" else 0, 1 if dtype == "fp8" else 0, B, Hq, hkv, dk, dv, scale, 1, None, None,
+               0, seed)
+    return _decode_multi(c, q, seq_lens, N, I, shard)
+
+
 def merge(O_part: np.ndarray, lse_part: np.ndarray):
     """LSE-weighted merge: O_part [N][B][H][Dv], lse_part [N][B][H] -> (O, lse)."""
     O_part = np.ascontiguousarray(O_part, dtype=np.float64)

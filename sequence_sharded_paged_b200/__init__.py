@@ -9,8 +9,9 @@ fallback: if the library is missing, importing the entry points raises.
 
 Entry points (same names as ``include/dcp.h``): ``dcp_shard_counts``,
 ``dcp_shard_map``, ``dcp_kv_append``, ``dcp_decode_workspace_size``,
-``dcp_decode_partial``, ``dcp_decode_partial_noalloc``, ``dcp_merge``,
-``dcp_get_device_status``.
+``dcp_decode_workspace_size_ex``, ``dcp_decode_partial``,
+``dcp_decode_partial_multi``, ``dcp_decode_merged``,
+``dcp_decode_partial_noalloc``, ``dcp_merge``, ``dcp_get_device_status``.
 """
 from __future__ import annotations
 
@@ -35,7 +36,8 @@ DCP_BF16 = 0
 DCP_FP8_E4M3 = 1
 
 EXPORTED = ("dcp_status_string", "dcp_shard_counts", "dcp_shard_map", "dcp_kv_append",
-            "dcp_decode_workspace_size", "dcp_decode_partial", "dcp_decode_partial_noalloc", "dcp_merge",
+            "dcp_decode_workspace_size", "dcp_decode_workspace_size_ex", "dcp_decode_partial",
+            "dcp_decode_partial_multi", "dcp_decode_merged", "dcp_decode_partial_noalloc", "dcp_merge",
             "dcp_get_device_status")
 
 
@@ -79,11 +81,16 @@ def lib() -> ctypes.CDLL:
         L.dcp_decode_workspace_size.argtypes = [D, i32]
         L.dcp_decode_workspace_size.restype = ctypes.c_size_t
         L.dcp_decode_partial.argtypes = [D, i32, P, P, P, P, P, ctypes.c_size_t, P]
+        L.dcp_decode_workspace_size_ex.argtypes = [D, i32, i32, i32]
+        L.dcp_decode_workspace_size_ex.restype = ctypes.c_size_t
+        L.dcp_decode_partial_multi.argtypes = [D, i32, i32, P, P, P, P, P, ctypes.c_size_t, P]
+        L.dcp_decode_merged.argtypes = [D, i32, i32, P, P, P, P, P, P, ctypes.c_size_t, P]
         L.dcp_decode_partial_noalloc.argtypes = [D, i32, P, P, P, P, P]
         L.dcp_merge.argtypes = [i32, i32, i32, i32, P, P, P, P, P]
         L.dcp_get_device_status.argtypes = [ctypes.POINTER(i32), P]
         for name in ("dcp_shard_counts", "dcp_shard_map", "dcp_kv_append", "dcp_decode_partial",
-                     "dcp_decode_partial_noalloc", "dcp_merge", "dcp_get_device_status"):
+                     "dcp_decode_partial_multi", "dcp_decode_merged", "dcp_decode_partial_noalloc", "dcp_merge",
+                     "dcp_get_device_status"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -144,6 +151,27 @@ def dcp_decode_partial(desc: CacheDesc, q, seq_lens, o_partial, lse, ws, stream=
     _check(lib().dcp_decode_partial(ctypes.byref(desc), q.shape[0], _ptr(q), _ptr(seq_lens), _ptr(o_partial),
                                     _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
            "dcp_decode_partial")
+
+
+def dcp_decode_workspace_size_ex(desc: CacheDesc, batch: int, q_len: int = 1, merged: bool = False) -> int:
+    return int(lib().dcp_decode_workspace_size_ex(ctypes.byref(desc), batch, q_len, 1 if merged else 0))
+
+
+def dcp_decode_partial_multi(desc: CacheDesc, q, seq_lens, o_partial, lse, ws, stream=None) -> None:
+    """q bf16 [B][q_len][hq][dk] -> o_partial [N][B][q_len][hq][dv], lse [N][B][q_len][hq]."""
+    _check(lib().dcp_decode_partial_multi(ctypes.byref(desc), q.shape[0], q.shape[1], _ptr(q), _ptr(seq_lens),
+                                          _ptr(o_partial), _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(),
+                                          _stream(stream)), "dcp_decode_partial_multi")
+
+
+def dcp_decode_merged(desc: CacheDesc, q, seq_lens, out, lse_out, ws, finish_ns=None, stream=None) -> None:
+    """Partial attention of every shard and the LSE merge in one launch sequence.
+    q bf16 [B][hq][dk] (one query token) or [B][q_len][hq][dk]; out / lse_out have
+    q's leading dimensions with dv / no trailing dimension; finish_ns int64 [B] or None."""
+    q_len = 1 if q.dim() == 3 else q.shape[1]
+    _check(lib().dcp_decode_merged(ctypes.byref(desc), q.shape[0], q_len, _ptr(q), _ptr(seq_lens), _ptr(out),
+                                   _ptr(lse_out), _ptr(finish_ns), _ptr(ws), ws.numel() * ws.element_size(),
+                                   _stream(stream)), "dcp_decode_merged")
 
 
 # size of the library's built-in decode scratch (DCP_STATIC_SCRATCH_BYTES in dcp.h)

@@ -132,7 +132,11 @@ struct Plan {
     DecodeGeometry g;
     WsLayout lay;
     size_t off_qs = 0, off_qinv = 0;  // fp8 MLA query split (0 when unused)
+    int q_len = 1;                    // query tokens per request (rows = q_len * hq)
+    int merged = 0;                   // 1: one output group per request
 };
+
+constexpr int kMaxQueryLen = 64;
 
 // The fp8 MLA kernel reads the query split into two e4m3 terms from the end of
 // the workspace: [B][128 rows][576] bytes + [B][64] fp32 reciprocals.
@@ -144,13 +148,25 @@ void add_query_split(const dcp_cache_desc* c, int B, Plan* p) {
     p->lay.total = align256(p->off_qinv + (size_t)B * 64 * sizeof(float));
 }
 
-bool make_plan(const dcp_cache_desc* c, int B, int num_sms, Plan* p) {
-    if (!decode_geometry(c->kind, c->dtype, c->hq, c->hkv, c->dk, c->dv, c->page_size, num_sms, &p->g)) return false;
+// Split slots: per-shard groups only split shards longer than one chunk, which
+// gives at most 2 * target + 2 slots; a merged group takes one slot per unit.
+int64_t split_bound(int64_t target, int64_t max_units, int merged) { return merged ? max_units : 2 * target + 2; }
+
+// The plan of a decode of B requests with q_len query tokens each (q_len * hq
+// query rows); merged != 0 gathers every shard of a request into one output
+// group.  Several query tokens are served by the tensor-core paths only.
+bool make_plan(const dcp_cache_desc* c, int B, int q_len, int merged, int num_sms, Plan* p) {
+    if (q_len < 1 || q_len > kMaxQueryLen) return false;
+    const int rows = q_len * c->hq;
+    if (!decode_geometry(c->kind, c->dtype, rows, c->hkv, c->dk, c->dv, c->page_size, num_sms, &p->g)) return false;
+    if (q_len > 1 && p->g.path != DecodePath::GqaMma && p->g.path != DecodePath::MlaUmma) return false;
     const int64_t target = (int64_t)p->g.units_per_cta * p->g.ctas;
     const int64_t max_units = (int64_t)c->n_shards * B + target + 1;
-    const int64_t max_split = 2 * target + 2;
+    const int64_t max_split = split_bound(target, max_units, merged);
     if (max_units > (1 << 30)) return false;
-    p->lay = ws_layout(c->n_shards, B, c->hq, c->dv, (int)max_units, (int)max_split);
+    p->lay = ws_layout(c->n_shards, B, rows, c->dv, (int)max_units, (int)max_split);
+    p->q_len = q_len;
+    p->merged = merged;
     add_query_split(c, B, p);
     return true;
 }
@@ -181,7 +197,7 @@ dcp_status decode_scratch(uint8_t** out) {
 // split slots), repeated down to one unit per CTA.  The bounds are make_plan's
 // for the smaller target.  False when nothing fits.
 bool make_plan_within(const dcp_cache_desc* c, int B, int num_sms, size_t cap, Plan* p) {
-    if (!make_plan(c, B, num_sms, p)) return false;
+    if (!make_plan(c, B, 1, 0, num_sms, p)) return false;
     while (p->lay.total > cap && p->g.units_per_cta > 1) {
         p->g.units_per_cta /= 2;
         const int64_t target = (int64_t)p->g.units_per_cta * p->g.ctas;
@@ -195,11 +211,13 @@ bool make_plan_within(const dcp_cache_desc* c, int B, int num_sms, size_t cap, P
 // The launch sequence of the decode (plan kernel, decode kernel) on a workspace
 // `w` laid out by `p`.
 dcp_status decode_on(const dcp_cache_desc* cache, int32_t B, const void* q, const int32_t* seq_lens,
-                     float* o_partial, float* lse, uint8_t* w, const Plan& p, int* status, cudaStream_t s) {
+                     float* o_partial, float* lse, uint8_t* w, const Plan& p, int* status, cudaStream_t s,
+                     int64_t* finish_ns = nullptr) {
     const int64_t target = (int64_t)p.g.units_per_cta * p.g.ctas;
-    cudaError_t e = launch_plan(seq_lens, B, cache->n_shards, cache->interleave, p.g.granule, p.g.min_chunk,
-                                (int)target, p.g.n_hb, w, p.lay.max_units, p.lay.max_split, cache->hq, cache->dv,
-                                status, s);
+    const int rows = p.q_len * cache->hq;
+    cudaError_t e = launch_plan(seq_lens, B, cache->n_shards, cache->interleave, p.q_len, p.merged, p.g.granule,
+                                p.g.min_chunk, (int)target, p.g.n_hb, w, p.lay.max_units, p.lay.max_split, rows,
+                                cache->dv, finish_ns, status, s);
     if (e != cudaSuccess) return DCP_ERR_CUDA;
     DecodeArgs a;
     a.k_pages = static_cast<const uint8_t*>(cache->k_pages);
@@ -212,7 +230,7 @@ dcp_status decode_on(const dcp_cache_desc* cache, int32_t B, const void* q, cons
     a.num_pages = cache->num_pages;
     a.batch = B;
     a.max_local_pages = cache->max_local_pages;
-    a.hq = cache->hq;
+    a.hq = rows;
     a.hkv = cache->hkv;
     a.dk = cache->dk;
     a.dv = cache->dv;
@@ -230,6 +248,8 @@ dcp_status decode_on(const dcp_cache_desc* cache, int32_t B, const void* q, cons
     a.qs = p.off_qs ? w + p.off_qs : nullptr;
     a.qinv = p.off_qinv ? reinterpret_cast<float*>(w + p.off_qinv) : nullptr;
     a.status = status;
+    a.q_len = p.q_len;
+    a.finish_ns = finish_ns;
     e = launch_decode(p.g, a, s);
     if (e == cudaErrorNotSupported) return DCP_ERR_UNSUPPORTED;
     return cuda_err(e);
@@ -391,7 +411,16 @@ size_t dcp_decode_workspace_size(const dcp_cache_desc* cache, int32_t B) {
     int num_sms = 0;
     if (device_info(nullptr, &num_sms) != DCP_OK) return 0;
     Plan p;
-    if (!make_plan(cache, B, num_sms, &p)) return 0;
+    if (!make_plan(cache, B, 1, 0, num_sms, &p)) return 0;
+    return p.lay.total;
+}
+
+size_t dcp_decode_workspace_size_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_len, int32_t merged) {
+    if (check_desc(cache, false) != DCP_OK || B != cache->batch) return 0;
+    int num_sms = 0;
+    if (device_info(nullptr, &num_sms) != DCP_OK) return 0;
+    Plan p;
+    if (!make_plan(cache, B, q_len, merged ? 1 : 0, num_sms, &p)) return 0;
     return p.lay.total;
 }
 
@@ -406,9 +435,42 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
     st = device_info(&status, &num_sms);
     if (st != DCP_OK) return st;
     Plan p;
-    if (!make_plan(cache, B, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
+    if (!make_plan(cache, B, 1, 0, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
     if (ws_bytes < p.lay.total) return DCP_ERR_WORKSPACE_TOO_SMALL;
     return decode_on(cache, B, q, seq_lens, o_partial, lse, static_cast<uint8_t*>(ws), p, status, (cudaStream_t)stream);
+}
+
+// Shared checks and launch of the two decode calls that take a query length.
+static dcp_status decode_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_len, int merged, const void* q,
+                            const int32_t* seq_lens, float* out, float* lse, int64_t* finish_ns, void* ws,
+                            size_t ws_bytes, void* stream) {
+    dcp_status st = check_desc(cache, true);
+    if (st != DCP_OK) return st;
+    if (B != cache->batch || q_len < 1 || !q || !seq_lens || !out || !lse || !ws) return DCP_ERR_INVALID_ARG;
+    if (q_len > kMaxQueryLen) return DCP_ERR_UNSUPPORTED;
+    if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || !aligned16(ws) || (finish_ns && !aligned16(finish_ns)))
+        return DCP_ERR_MISALIGNED;
+    int* status = nullptr;
+    int num_sms = 0;
+    st = device_info(&status, &num_sms);
+    if (st != DCP_OK) return st;
+    Plan p;
+    if (!make_plan(cache, B, q_len, merged, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
+    if (ws_bytes < p.lay.total) return DCP_ERR_WORKSPACE_TOO_SMALL;
+    return decode_on(cache, B, q, seq_lens, out, lse, static_cast<uint8_t*>(ws), p, status, (cudaStream_t)stream,
+                     finish_ns);
+}
+
+dcp_status dcp_decode_partial_multi(const dcp_cache_desc* cache, int32_t B, int32_t q_len, const void* q,
+                                    const int32_t* seq_lens, float* o_partial, float* lse, void* ws, size_t ws_bytes,
+                                    void* stream) {
+    return decode_ex(cache, B, q_len, 0, q, seq_lens, o_partial, lse, nullptr, ws, ws_bytes, stream);
+}
+
+dcp_status dcp_decode_merged(const dcp_cache_desc* cache, int32_t B, int32_t q_len, const void* q,
+                             const int32_t* seq_lens, float* out, float* lse_out, int64_t* finish_ns, void* ws,
+                             size_t ws_bytes, void* stream) {
+    return decode_ex(cache, B, q_len, 1, q, seq_lens, out, lse_out, finish_ns, ws, ws_bytes, stream);
 }
 
 // No workspace argument and no allocation: for callers that cannot allocate
@@ -427,7 +489,7 @@ dcp_status dcp_decode_partial_noalloc(const dcp_cache_desc* cache, int32_t B, co
     st = device_info(&status, &num_sms);
     if (st != DCP_OK) return st;
     Plan p;
-    if (!make_plan(cache, B, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
+    if (!make_plan(cache, B, 1, 0, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
     if (!make_plan_within(cache, B, num_sms, DCP_STATIC_SCRATCH_BYTES, &p)) return DCP_ERR_WORKSPACE_TOO_SMALL;
     uint8_t* w = nullptr;
     st = decode_scratch(&w);

@@ -162,10 +162,12 @@ struct Unit {
     int32_t n;          // shard
     int32_t b;          // request
     int32_t t0, t1;     // local token range [t0, t1) of shard n of request b
-    int32_t slot;       // split-partial slot of this chunk, -1 when the shard is one chunk
-    int32_t n_chunks;   // chunks of this shard
-    int32_t slot_base;  // first split slot of this shard
-    int32_t pad;
+    int32_t slot;       // split-partial slot of this unit, -1 when its group has one unit
+    int32_t n_chunks;   // units of this unit's output group
+    int32_t slot_base;  // first split slot of the group
+    int32_t grp;        // output group: row block grp of the outputs (n*B + b for per-shard
+                        // partials, b for the merged output); the group's last unit to finish
+                        // LSE-merges its units' split partials there
 };
 static_assert(sizeof(Unit) == 32, "Unit layout");
 
@@ -176,7 +178,8 @@ struct PlanHeader {
     int32_t max_split;
     int64_t total_tokens;
     int32_t next_unit;  // dynamic-scheduling ticket (zeroed by the planner)
-    int32_t pad;
+    int32_t merged;     // 1: one output group per request (all shards merged)
+    int64_t t_start_ns; // %globaltimer when the planner started
 };
 
 // Per-stage metadata of the dynamically scheduled kernels: which unit and
@@ -252,7 +255,34 @@ struct DecodeArgs {
     uint8_t* qs;         // fp8 MLA: query rows split into two e4m3 terms [B][128][576] (else null)
     float* qinv;         // fp8 MLA: 1 / sigma per (request, head) [B][64] (else null)
     int* status;
+    // several query tokens per request: hq counts query ROWS (q_len x heads), row
+    // r = j * (hq / q_len) + head belongs to query token j
+    int32_t q_len;
+    int64_t* finish_ns;  // per output group: ns from the planner's start to its final output (or null)
 };
+
+// Local tokens [0, limit) of shard u.n that query token j attends: the positions
+// p <= L_b - q_len + j (causal among the q_len new tokens, which are the last
+// positions of the request).  With one query token every owned token is attended.
+__device__ __forceinline__ int row_limit(const DecodeArgs& a, const Unit& u, int j) {
+    if (a.q_len <= 1) return 0x7fffffff;
+    const int L = __ldg(a.seq_lens + u.b) - a.q_len + j + 1;
+    return L <= 0 ? 0 : (int)count_of(L, a.n_shards, a.interleave, u.n);
+}
+
+// Completion time of output group `grp` (call after a part of its final output
+// is stored; the planner zeroes the array and the last part to finish sets it).
+__device__ __forceinline__ void record_finish(const DecodeArgs& a, int grp) {
+    if (!a.finish_ns) return;
+    const uint64_t dt = global_timer_ns() - (uint64_t)a.plan->t_start_ns;
+    atomicMax(reinterpret_cast<unsigned long long*>(a.finish_ns + grp), (unsigned long long)dt);
+}
+
+// Invalidate the 128-byte L2 line at p (128-byte aligned) without writing it
+// back: for scratch data that has been read for the last time.
+__device__ __forceinline__ void discard_l2_line(const void* p) {
+    asm volatile("discard.global.L2 [%0], 128;" ::"l"(p) : "memory");
+}
 
 // Fetch the physical page of local page j of (n, b); -1 when invalid.
 __device__ __forceinline__ int page_of(const DecodeArgs& a, int n, int b, int j) {

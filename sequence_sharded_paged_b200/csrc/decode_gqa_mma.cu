@@ -85,7 +85,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
     float* sM = sO + a.hq * D;                                                   // [NCW][16]
     float* sL = sM + NCW * 16;                                                   // [NCW][16]
     float* sLse = sL + NCW * 16;                                                 // [hq]
-    uint64_t* full = reinterpret_cast<uint64_t*>(sLse + a.hq + (a.hq & 1));
+    float* sTot = sLse + a.hq;                                                   // [hq]
+    uint64_t* full = reinterpret_cast<uint64_t*>(sTot + a.hq + (a.hq & 1));
     uint64_t* empty = full + stages;
     StageMeta* smeta = reinterpret_cast<StageMeta*>(empty + stages);
     __shared__ int s_flag;
@@ -183,12 +184,19 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
     const int g = warp % hkv;
     const int r = warp / hkv;
     const int qr = lane >> 2, qc = lane & 3;  // quad row / column
+    // The 16 MMA rows of KV head g: with q_len query tokens per request, row r is
+    // query token r / G of head g * G + r % G (G = heads per KV head); its output
+    // row is (r / G) * (query heads) + g * G + r % G.
+    const int G = 16 / a.q_len;
+    const int hq_heads = a.hq / a.q_len;
+    auto orow = [&](int gg, int rr) { return (rr / G) * hq_heads + gg * G + (rr % G); };
     const uint32_t ring_u32 = smem_u32(ring);
     int stage = 0;
     uint32_t phase = 0;
     uint32_t qa[D / 16][4];
     float o[D / 8][4];
     float m0 = -INFINITY, m1 = -INFINITY, l0 = 0.f, l1 = 0.f;
+    int lim0 = 0x7fffffff, lim1 = 0x7fffffff;  // causal limits of rows qr and qr + 8
     Unit u = a.units[0];
     while (true) {
         if (!mbar_wait(full + stage, phase, &s_abort, a.status)) break;
@@ -196,15 +204,18 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
         if (meta.unit < 0) break;
         if (meta.flags & kStageFirst) {
             u = a.units[meta.unit];
-            // Q fragments (A operand), 16 heads x D
-            const uint32_t* q32 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)u.b * a.hq + g * 16) * D);
+            // Q fragments (A operand), 16 rows x D
+            const uint32_t* q0 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)u.b * a.hq + orow(g, qr)) * D);
+            const uint32_t* q1 = reinterpret_cast<const uint32_t*>(a.q + ((int64_t)u.b * a.hq + orow(g, qr + 8)) * D);
 #pragma unroll
             for (int kk = 0; kk < D / 16; kk++) {
-                qa[kk][0] = __ldg(q32 + (qr * D + kk * 16 + 2 * qc) / 2);
-                qa[kk][1] = __ldg(q32 + ((qr + 8) * D + kk * 16 + 2 * qc) / 2);
-                qa[kk][2] = __ldg(q32 + (qr * D + kk * 16 + 8 + 2 * qc) / 2);
-                qa[kk][3] = __ldg(q32 + ((qr + 8) * D + kk * 16 + 8 + 2 * qc) / 2);
+                qa[kk][0] = __ldg(q0 + (kk * 16 + 2 * qc) / 2);
+                qa[kk][1] = __ldg(q1 + (kk * 16 + 2 * qc) / 2);
+                qa[kk][2] = __ldg(q0 + (kk * 16 + 8 + 2 * qc) / 2);
+                qa[kk][3] = __ldg(q1 + (kk * 16 + 8 + 2 * qc) / 2);
             }
+            lim0 = row_limit(a, u, qr / G);
+            lim1 = row_limit(a, u, (qr + 8) / G);
 #pragma unroll
             for (int i = 0; i < D / 8; i++) o[i][0] = o[i][1] = o[i][2] = o[i][3] = 0.f;
             m0 = m1 = -INFINITY;
@@ -231,14 +242,15 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
                     mma_bf16(s[0], qa[kk], b0, b1);
                     mma_bf16(s[1], qa[kk], b2, b3);
                 }
-                // online softmax (log2 domain); rows qr and qr + 8
+                // online softmax (log2 domain); rows qr and qr + 8, each cut by its causal limit
+                const int nv0 = min(nvalid, max(0, lim0 - t)), nv1 = min(nvalid, max(0, lim1 - t));
                 float x[2][4];
 #pragma unroll
                 for (int nt = 0; nt < 2; nt++)
 #pragma unroll
                     for (int e = 0; e < 4; e++) {
                         const int tok = nt * 8 + 2 * qc + (e & 1);
-                        x[nt][e] = tok < nvalid ? s[nt][e] * a.scale_log2 : -INFINITY;
+                        x[nt][e] = tok < (e < 2 ? nv0 : nv1) ? s[nt][e] * a.scale_log2 : -INFINITY;
                     }
                 float mx0 = fmaxf(fmaxf(x[0][0], x[0][1]), fmaxf(x[1][0], x[1][1]));
                 float mx1 = fmaxf(fmaxf(x[0][2], x[0][3]), fmaxf(x[1][2], x[1][3]));
@@ -345,8 +357,8 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
             if (r == k) {
 #pragma unroll
                 for (int i = 0; i < D / 8; i++) {
-                    float* row0 = sO + (g * 16 + qr) * D + i * 8 + 2 * qc;
-                    float* row1 = sO + (g * 16 + qr + 8) * D + i * 8 + 2 * qc;
+                    float* row0 = sO + orow(g, qr) * D + i * 8 + 2 * qc;
+                    float* row1 = sO + orow(g, qr + 8) * D + i * 8 + 2 * qc;
                     if (k == 0) {
                         row0[0] = o[i][0] * w0;
                         row0[1] = o[i][1] * w0;
@@ -365,17 +377,19 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
         // normalise and LSE (natural log)
         const int tid = threadIdx.x;
         for (int i = tid; i < a.hq; i += NT) {
-            const int gg = i / 16, row = i % 16;
+            // output row i = (query token j, head hh): KV head hh / G, MMA row j * G + hh % G
+            const int j = i / hq_heads, hh = i - j * hq_heads;
+            const int gg = hh / G, row = j * G + hh % G;
             float M = -INFINITY, Ls = 0.f;
             for (int k = 0; k < R; k++) M = fmaxf(M, sM[(k * hkv + gg) * 16 + row]);
             for (int k = 0; k < R; k++) Ls += sL[(k * hkv + gg) * 16 + row];
             sLse[i] = (M == -INFINITY || Ls == 0.f) ? -INFINITY : (M + log2f(Ls)) * kLn2;
-            sL[i % 16 + (i / 16) * 16] = Ls;  // reuse: total per head
+            sTot[i] = Ls;
         }
         named_barrier_sync(1, NT);
         for (int i = tid; i < a.hq * D; i += NT) {
             const int h = i / D;
-            const float Ls = sL[h];
+            const float Ls = sTot[h];
             sO[i] = Ls > 0.f ? sO[i] / Ls : 0.f;
         }
         named_barrier_sync(1, NT);
@@ -387,7 +401,7 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
 template <int D, int NCW>
 size_t gqa_mma_smem(int hq, int hkv, int stages) {
     const size_t stage_bytes = (size_t)hkv * 2 * (D / 64) * kBoxBytes;
-    return 1024 + (size_t)stages * stage_bytes + (size_t)(hq * D + 2 * NCW * 16 + hq + 2) * 4 +
+    return 1024 + (size_t)stages * stage_bytes + (size_t)(hq * D + 2 * NCW * 16 + 2 * hq + 2) * 4 +
            (size_t)2 * stages * 8 + (size_t)stages * sizeof(StageMeta);
 }
 

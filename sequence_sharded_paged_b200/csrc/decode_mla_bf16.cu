@@ -312,10 +312,11 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
         uint32_t seq = 0, unit_k = 0;
         float m_used = -INFINITY, lsum = 0.f;
+        int lim = 0x7fffffff;  // local tokens [0, lim) of the unit's shard this row attends
         bool o_has = false;
         bool fail = false;
         Unit u;
-        u.n = u.b = u.t0 = u.t1 = u.slot = u.n_chunks = u.slot_base = u.pad = 0;
+        u.n = u.b = u.t0 = u.t1 = u.slot = u.n_chunks = u.slot_base = u.grp = 0;
         while (true) {
             const int ts = seq & 1;
             const uint32_t par = (seq >> 1) & 1;
@@ -330,6 +331,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nvalid = (meta.flags >> 8) & 0xFF;
             if (first) {
                 u = a.units[meta.unit];
+                lim = head ? row_limit(a, u, h / (HQ / a.q_len)) : 0x7fffffff;
                 // Q of request u.b: all S MMAs of the previous unit are complete (first unit passes)
                 fail = !mbar_wait(bar + B_Q_FREE, (unit_k & 1) ^ 1, s_abort, a.status);
                 if (!fail) {
@@ -351,6 +353,9 @@ __global__ void __launch_bounds__(kThreads, 1)
             if (!fail) fail = !mbar_wait(bar + B_S_FULL + ts, par, s_abort, a.status);
             if (threadIdx.x == 64) TRACE(6, seq);
             umma::fence_after_sync();
+            // tokens of the tile this row attends: the tile's valid tokens, cut by the row's
+            // causal limit when the request has several query tokens
+            const int row_nv = min(nvalid, max(0, lim - meta.t));
             float x[32];
             {
                 uint32_t v0[32], v1[32];
@@ -361,7 +366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                 for (int j = 0; j < 32; j++) {
                     const uint32_t recv = __shfl_xor_sync(0xffffffffu, v1[j], 16);
                     const float v = __uint_as_float(half ? recv : v0[j]);
-                    x[j] = base + j < nvalid ? v * a.scale_log2 : -INFINITY;
+                    x[j] = base + j < row_nv ? v * a.scale_log2 : -INFINITY;
                 }
             }
             float mt = -INFINITY;
@@ -456,10 +461,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float l = lsum + __shfl_xor_sync(0xffffffffu, lsum, 16);  // both halves of the head
                 if (head && half == 0) s_l[h] = l > 0.f ? 1.f / l : 0.f;      // O = O^T * (1 / l)
                 if (named_barrier_or(kSmBar, 128, fail)) break;
-                const int64_t shard = (int64_t)u.n * a.batch + u.b;
+                const int64_t grp = u.grp;
                 const bool split = u.n_chunks > 1;
-                float* obase = split ? a.split_o + (int64_t)u.slot * a.hq * 512 : a.o_partial + shard * a.hq * 512;
-                float* lbase = split ? a.split_lse + (int64_t)u.slot * a.hq : a.lse + shard * a.hq;
+                float* obase = split ? a.split_o + (int64_t)u.slot * a.hq * 512 : a.o_partial + grp * a.hq * 512;
+                float* lbase = split ? a.split_lse + (int64_t)u.slot * a.hq : a.lse + grp * a.hq;
 #pragma unroll 1
                 for (int blk = 0; blk < 4; blk++) {
                     const int dv = blk * 128 + 32 * qd + lane;
@@ -478,17 +483,24 @@ __global__ void __launch_bounds__(kThreads, 1)
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar + B_O_FREE);
                 if (split) {
-                    // split-KV reduce: the last chunk of the shard to finish merges the chunks
+                    // the last unit of the group to finish merges the group's split partials
                     __threadfence();
                     named_barrier_sync(kSmBar, 128);
-                    if (tid == 0) s_misc[2] = (atomicAdd(a.done + shard, 1) == u.n_chunks - 1) ? 1 : 0;
+                    if (tid == 0) s_misc[2] = (atomicAdd(a.done + grp, 1) == u.n_chunks - 1) ? 1 : 0;
                     named_barrier_sync(kSmBar, 128);
                     const int is_last = *reinterpret_cast<volatile int*>(s_misc + 2);
                     named_barrier_sync(kSmBar, 128);
                     if (is_last) {
                         __threadfence();
-                        merge_split_chunks(a, u, shard, 0, HQ, tid, 128);
+                        merge_split_chunks(a, u, 0, HQ, tid, 128, kSmBar);
+                        if (a.finish_ns) {
+                            named_barrier_sync(kSmBar, 128);
+                            if (tid == 0) record_finish(a, (int)grp);
+                        }
                     }
+                } else if (a.finish_ns) {
+                    named_barrier_sync(kSmBar, 128);
+                    if (tid == 0) record_finish(a, (int)grp);
                 }
             }
             seq++;

@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (lane == 0) tma_prefetch_desc(&tmC);
         int ui = -1, k = 0, nt = 0;
         Unit u;
-        u.n = u.b = u.t0 = u.t1 = u.slot = u.n_chunks = u.slot_base = u.pad = 0;
+        u.n = u.b = u.t0 = u.t1 = u.slot = u.n_chunks = u.slot_base = u.grp = 0;
         // moves (ui, k) to the next page (the same on every lane); false when no work is left
         auto advance = [&]() -> bool {
             if (ui >= 0 && k + 1 < nt) {
@@ -468,9 +468,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         const uint32_t lane_off = (uint32_t)(32 * qd) << 16;
         uint32_t seq = 0, kk = 0, unit_k = 0;
         float m_used = -INFINITY, lpart = 0.f, f = 0.f;
+        int lim = 0x7fffffff;  // local tokens [0, lim) of the unit's shard this row attends
         bool o_has = false, fail = false;
         Unit u;
-        u.n = u.b = u.t0 = u.t1 = u.slot = u.n_chunks = u.slot_base = u.pad = 0;
+        u.n = u.b = u.t0 = u.t1 = u.slot = u.n_chunks = u.slot_base = u.grp = 0;
         while (true) {
             const int pb = seq & 1;
             const int slot0 = slot_of(kk);
@@ -490,10 +491,11 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool mine = wg == 0 || pair;          // does my page exist in this tile
             const int my_slot = mine ? slot0 + wg : slot0;
             const int nvalid = mine ? (((wg ? m1.flags : m0.flags) >> 8) & 0xFF) : 0;
-            const bool full = nvalid == kPg;
+            const bool page_full = nvalid == kPg;
             if (first) {
                 u = a.units[m0.unit];
                 f = head ? __ldg(a.qinv + (int64_t)u.b * 64 + h) * a.scale_log2 : 0.f;
+                lim = head ? row_limit(a, u, h / (HQ / a.q_len)) : 0x7fffffff;
                 // the previous unit's S MMAs are complete (first unit passes at once)
                 fail = fail || !mbar_wait(bar + B_Q_FREE, (unit_k & 1) ^ 1, s_abort, a.status);
                 if (!fail) {
@@ -534,6 +536,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 lpart = 0.f;
                 o_has = false;
             }
+            // tokens of my page this row attends: the page's valid tokens, cut by the row's
+            // causal limit when the request has several query tokens
+            const int row_nv = min(nvalid, max(0, lim - (wg ? m1.t : m0.t)));
+            const bool full = row_nv == kPg;
             // ---- scores of my page: rows S_hi (lane < 16) and S_lo (lane >= 16) of head h; swap halves
             if (!fail) fail = !mbar_wait(bar + B_S_FULL, seq & 1, s_abort, a.status);
             umma::fence_after_sync();
@@ -575,7 +581,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                         const float sc[4] = {sc4.x, sc4.y, sc4.z, sc4.w};
 #pragma unroll
                         for (int e = 0; e < 4; e++) {
-                            const bool valid = base + 4 * j4 + e < nvalid;
+                            const bool valid = base + 4 * j4 + e < row_nv;
                             x[4 * j4 + e] = valid ? x[4 * j4 + e] : -INFINITY;
                             smax = valid ? fmaxf(smax, sc[e]) : smax;
                         }
@@ -653,7 +659,7 @@ __global__ void __launch_bounds__(kThreads, 1)
                     }
                     if (!full) {
 #pragma unroll
-                        for (int j = 0; j < 32; j++) w[j] = (base + j < nvalid) ? w[j] : 0.f;
+                        for (int j = 0; j < 32; j++) w[j] = (base + j < row_nv) ? w[j] : 0.f;
                     }
                 } else {
 #pragma unroll
@@ -675,7 +681,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             } else if (!fail) {
                 lpart = lpart * alpha;
             }
-            if (!fail && mine && !full) {
+            if (!fail && mine && !page_full) {
                 // rows past the last valid token hold stale page bytes (possibly NaN codes):
                 // zero their value columns so that W = 0 cannot meet them (token group wg
                 // clears its own page)
@@ -701,10 +707,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma::fence_after_sync();
                 const float lg = lpart + __shfl_xor_sync(0xffffffffu, lpart, 16);  // this token group
                 if (half == 0) s_gl[wg * 64 + h] = lg;
-                const int64_t shard = (int64_t)u.n * a.batch + u.b;
+                const int64_t grp = u.grp;
                 const bool split = u.n_chunks > 1;
-                float* obase = split ? a.split_o + (int64_t)u.slot * a.hq * 512 : a.o_partial + shard * a.hq * 512;
-                float* lbase = split ? a.split_lse + (int64_t)u.slot * a.hq : a.lse + shard * a.hq;
+                float* obase = split ? a.split_o + (int64_t)u.slot * a.hq * 512 : a.o_partial + grp * a.hq * 512;
+                float* lbase = split ? a.split_lse + (int64_t)u.slot * a.hq : a.lse + grp * a.hq;
                 if (named_barrier_or(kSmBar, 256, fail)) break;
                 if (head && half == 0 && wg == 0) {
                     const float l = lg + s_gl[64 + h];
@@ -734,14 +740,21 @@ __global__ void __launch_bounds__(kThreads, 1)
                 if (split) {
                     __threadfence();
                     named_barrier_sync(kSmBar, 256);
-                    if (tid == 0) s_misc[2] = (atomicAdd(a.done + shard, 1) == u.n_chunks - 1) ? 1 : 0;
+                    if (tid == 0) s_misc[2] = (atomicAdd(a.done + grp, 1) == u.n_chunks - 1) ? 1 : 0;
                     named_barrier_sync(kSmBar, 256);
                     const int is_last = *reinterpret_cast<volatile int*>(s_misc + 2);
                     named_barrier_sync(kSmBar, 256);
                     if (is_last) {
                         __threadfence();
-                        merge_split_chunks(a, u, shard, 0, HQ, tid, 256);
+                        merge_split_chunks(a, u, 0, HQ, tid, 256, kSmBar);
+                        if (a.finish_ns) {
+                            named_barrier_sync(kSmBar, 256);
+                            if (tid == 0) record_finish(a, (int)grp);
+                        }
                     }
+                } else if (a.finish_ns) {
+                    named_barrier_sync(kSmBar, 256);
+                    if (tid == 0) record_finish(a, (int)grp);
                 }
                 if (threadIdx.x == 64) TRACE(13, seq);
             }

@@ -33,10 +33,11 @@ cudaError_t launch_shard_map(int64_t n_pos, const int32_t* pos, const int32_t* r
                              int32_t* local_out, int64_t* slot_out, int* status, cudaStream_t s);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 
-// planner: splits every (shard, request) into chunks of at most chunk_tokens
-cudaError_t launch_plan(const int32_t* seq_lens, int B, int N, int I, int granule, int min_chunk, int target_units,
-                        int n_hb, void* ws, int max_units, int max_split, int hq, int dv, int* status,
-                        cudaStream_t s);
+// planner: splits every (shard, request) into chunks of at most chunk_tokens and
+// gathers them into output groups (per shard, or per request when merged != 0)
+cudaError_t launch_plan(const int32_t* seq_lens, int B, int N, int I, int q_len, int merged, int granule,
+                        int min_chunk, int target_units, int n_hb, void* ws, int max_units, int max_split, int hq,
+                        int dv, int64_t* finish_ns, int* status, cudaStream_t s);
 
 // decode kernels; each returns cudaErrorNotSupported for shapes it does not cover
 enum class DecodePath { GqaSimt, GqaMma, MlaSimt, MlaUmma };

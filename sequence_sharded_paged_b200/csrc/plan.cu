@@ -1,12 +1,22 @@
-// plan.cu -- split-KV work planner for dcp_decode_partial.
+// plan.cu -- split-KV work planner for the decode calls.
 //
 // Every (shard n, request b) owns count_n(L_b) local tokens.  The planner cuts
 // each into chunks of at most C tokens (C a multiple of the kernel's token
 // granule, at least total_tokens / target_units), so the persistent decode
 // grid sees many similar-sized units regardless of the length mix, and lists
-// the units longest-first (bucketed by floor(log2(length))).  Shards cut into
-// several chunks get consecutive split-partial slots; the last chunk of such a
-// shard to finish merges them (same LSE arithmetic as dcp_merge).
+// the units longest-first (bucketed by floor(log2(length))).
+//
+// Units are gathered into output groups; a group with several units gives each
+// a split-partial slot and its last unit to finish LSE-merges them (the
+// arithmetic of "Efficient Decode Context Parallelism with vLLM for Long
+// Context Workloads", section 4.1, which the all-gather + reduce-scatter of
+// the pages performs across GPUs):
+//  - per-shard partials: one group per (n, b), output row block n*B + b;
+//  - merged output: one group per request b over the chunks of ALL its shards,
+//    output row block b.  The group's units are listed next to each other, so
+//    they run at the same time on different SMs and the merging unit finds
+//    their partials still in L2.  Empty shards add no unit; a request with no
+//    token at all gets one empty unit (O = 0, LSE = -inf).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -47,13 +57,14 @@ __device__ int block_scan_incl(int v, int* total, int* warp_sums) {
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ seq_lens, int B, int N, int I,
-                                                            int granule, int min_chunk, int target_units,
-                                                            int n_hb, uint8_t* ws, WsLayout lay, int* status) {
+                                                            int q_len, int merged, int granule, int min_chunk,
+                                                            int target_units, int n_hb, uint8_t* ws, WsLayout lay,
+                                                            int64_t* finish_ns, int* status) {
     PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws);
     Unit* units = reinterpret_cast<Unit*>(ws + lay.off_units);
     int32_t* done = reinterpret_cast<int32_t*>(ws + lay.off_done);
-    int32_t* shard_k = reinterpret_cast<int32_t*>(ws + lay.off_k);
-    int32_t* slot_base = reinterpret_cast<int32_t*>(ws + lay.off_base);
+    int32_t* grp_k = reinterpret_cast<int32_t*>(ws + lay.off_k);       // units per group [groups]
+    int32_t* slot_base = reinterpret_cast<int32_t*>(ws + lay.off_base);  // [groups]
 
     __shared__ unsigned long long s_total;
     __shared__ int s_hist[33];
@@ -63,6 +74,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     __shared__ int s_split_total;
     const int tid = threadIdx.x;
     if (tid == 0) {
+        hdr->t_start_ns = (int64_t)global_timer_ns();
         s_total = 0;
         s_units_total = 0;
         s_split_total = 0;
@@ -74,7 +86,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     unsigned long long t = 0;
     for (int b = tid; b < B; b += kPlanThreads) {
         int L = seq_lens[b];
-        if (L < 0) record_status(status, DCP_ERR_INVALID_ARG);
+        if (L < 0 || (L > 0 && L < q_len)) record_status(status, DCP_ERR_INVALID_ARG);
         t += (unsigned long long)(L < 0 ? 0 : L);
     }
     atomicAdd(&s_total, t);
@@ -87,32 +99,47 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     C = (C + granule - 1) / granule * granule;
     if (C > (1 << 30)) C = 1 << 30;
 
-    // 3. chunks per shard, split-slot scan, length histogram
-    const int NB = N * B;
-    for (int i = tid; i < NB * n_hb; i += kPlanThreads) done[i] = 0;
+    // 3. units per group, split-slot scan, length histogram (a group's units share
+    //    one bucket in merged mode: that of its longest unit)
+    const int NG = merged ? B : N * B;
+    for (int i = tid; i < NG * n_hb; i += kPlanThreads) done[i] = 0;
+    if (finish_ns)
+        for (int i = tid; i < NG; i += kPlanThreads) finish_ns[i] = 0;
     int units_local = 0;
     int carry = 0;
-    for (int base = 0; base < NB; base += kPlanThreads) {
-        int s = base + tid;
+    for (int base = 0; base < NG; base += kPlanThreads) {
+        const int gi = base + tid;
         int k = 0, split = 0;
-        if (s < NB) {
-            int n = s / B, b = s - n * B;
-            int L = seq_lens[b];
-            int64_t cnt = count_of(L < 0 ? 0 : L, N, I, n);
-            k = cnt == 0 ? 1 : (int)((cnt + C - 1) / C);
-            shard_k[s] = k;
+        if (gi < NG) {
+            if (merged) {
+                const int L = max(seq_lens[gi], 0);
+                int64_t cmax = 0;
+                for (int n = 0; n < N; n++) {
+                    const int64_t cnt = count_of(L, N, I, n);
+                    k += (int)((cnt + C - 1) / C);
+                    cmax = cnt > cmax ? cnt : cmax;
+                }
+                if (k == 0) k = 1;
+                atomicAdd(&s_hist[cmax > 0 ? length_bucket(cmax < C ? cmax : C) : 32], k);
+            } else {
+                const int n = gi / B, b = gi - n * B;
+                const int L = seq_lens[b];
+                const int64_t cnt = count_of(L < 0 ? 0 : L, N, I, n);
+                k = cnt == 0 ? 1 : (int)((cnt + C - 1) / C);
+                if (cnt > 0) {
+                    if (k > 1) atomicAdd(&s_hist[length_bucket(C)], k - 1);
+                    atomicAdd(&s_hist[length_bucket(cnt - (int64_t)(k - 1) * C)], 1);
+                } else {
+                    atomicAdd(&s_hist[32], 1);
+                }
+            }
+            grp_k[gi] = k;
             split = k >= 2 ? k : 0;
             units_local += k;
-            if (cnt > 0) {
-                if (k > 1) atomicAdd(&s_hist[length_bucket(C)], k - 1);
-                atomicAdd(&s_hist[length_bucket(cnt - (int64_t)(k - 1) * C)], 1);
-            } else {
-                atomicAdd(&s_hist[32], 1);
-            }
         }
         int total;
         int incl = block_scan_incl(split, &total, s_warp);
-        if (s < NB) slot_base[s] = carry + incl - split;
+        if (gi < NG) slot_base[gi] = carry + incl - split;
         carry += total;
     }
     atomicAdd(&s_units_total, units_local);
@@ -135,16 +162,54 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
         hdr->max_split = lay.max_split;
         hdr->total_tokens = T;
         hdr->next_unit = 0;
+        hdr->merged = merged;
         if (!fits) record_status(status, DCP_ERR_WORKSPACE_TOO_SMALL);
     }
     if (!fits) return;
 
     // 4. emit units, longest bucket first
-    for (int s = tid; s < NB; s += kPlanThreads) {
+    if (merged) {
+        for (int b = tid; b < B; b += kPlanThreads) {
+            const int L = max(seq_lens[b], 0);
+            const int k = grp_k[b];
+            const int sb = slot_base[b];
+            int64_t cmax = 0;
+            for (int n = 0; n < N; n++) {
+                const int64_t cnt = count_of(L, N, I, n);
+                cmax = cnt > cmax ? cnt : cmax;
+            }
+            int pos = atomicAdd(&s_cursor[cmax > 0 ? length_bucket(cmax < C ? cmax : C) : 32], k);
+            Unit u;
+            u.b = b;
+            u.n_chunks = k;
+            u.slot_base = k >= 2 ? sb : -1;
+            u.grp = b;
+            if (cmax == 0) {  // a request with no token: one empty unit
+                u.n = 0;
+                u.t0 = u.t1 = 0;
+                u.slot = -1;
+                units[pos] = u;
+                continue;
+            }
+            int j = 0;
+            for (int n = 0; n < N; n++) {
+                const int64_t cnt = count_of(L, N, I, n);
+                for (int64_t t0 = 0; t0 < cnt; t0 += C, j++) {
+                    u.n = n;
+                    u.t0 = (int32_t)t0;
+                    u.t1 = (int32_t)(t0 + C < cnt ? t0 + C : cnt);
+                    u.slot = k >= 2 ? sb + j : -1;
+                    units[pos + j] = u;
+                }
+            }
+        }
+        return;
+    }
+    for (int s = tid; s < NG; s += kPlanThreads) {
         int n = s / B, b = s - n * B;
         int L = seq_lens[b];
         int64_t cnt = count_of(L < 0 ? 0 : L, N, I, n);
-        int k = shard_k[s];
+        int k = grp_k[s];
         int sb = slot_base[s];
         for (int j = 0; j < k; j++) {
             int64_t t0 = (int64_t)j * C;
@@ -158,7 +223,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
             u.slot = k >= 2 ? sb + j : -1;
             u.n_chunks = k;
             u.slot_base = k >= 2 ? sb : -1;
-            u.pad = 0;
+            u.grp = s;
             units[pos] = u;
         }
     }
@@ -166,12 +231,12 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
 
 }  // namespace
 
-cudaError_t launch_plan(const int32_t* seq_lens, int B, int N, int I, int granule, int min_chunk, int target_units,
-                        int n_hb, void* ws, int max_units, int max_split, int hq, int dv, int* status,
-                        cudaStream_t s) {
+cudaError_t launch_plan(const int32_t* seq_lens, int B, int N, int I, int q_len, int merged, int granule,
+                        int min_chunk, int target_units, int n_hb, void* ws, int max_units, int max_split, int hq,
+                        int dv, int64_t* finish_ns, int* status, cudaStream_t s) {
     WsLayout lay = ws_layout(N, B, hq, dv, max_units, max_split);
-    plan_kernel<<<1, kPlanThreads, 0, s>>>(seq_lens, B, N, I, granule, min_chunk, target_units, n_hb,
-                                           reinterpret_cast<uint8_t*>(ws), lay, status);
+    plan_kernel<<<1, kPlanThreads, 0, s>>>(seq_lens, B, N, I, q_len, merged, granule, min_chunk, target_units, n_hb,
+                                           reinterpret_cast<uint8_t*>(ws), lay, finish_ns, status);
     return cudaGetLastError();
 }
 

@@ -29,8 +29,8 @@ def _rank_main(rank, world, port, q):
     dist.init_process_group("gloo", rank=rank, world_size=world)
     try:
         # rank r: device time 10 + r ms, kernel time 5 + 2r, e2e 20 - r; bytes 1000 (r + 1)
-        out = bench.combine_ranks(dist, torch.device("cpu"), 10.0 + rank, 5.0 + 2 * rank, 20.0 - rank,
-                                  1000 * (rank + 1), 7 * (rank + 1))
+        out = bench.combine_ranks(dist, torch.device("cpu"), [10.0 + rank, 5.0 + 2 * rank, 20.0 - rank],
+                                  [1000 * (rank + 1), 7 * (rank + 1)])
         q.put((rank, out))
     finally:
         dist.destroy_process_group()
@@ -48,7 +48,7 @@ def test_combine_ranks_two_gloo_ranks():
         p.join(timeout=60)
         assert p.exitcode == 0
     for r in (0, 1):
-        ms, kern, e2e, b, eb = res[r]
+        (ms, kern, e2e), (b, eb) = res[r]
         assert ms == 11.0 and kern == 7.0 and e2e == 20.0  # max over ranks
         assert b == 3000.0 and eb == 21.0                 # sum over ranks
 
@@ -73,9 +73,25 @@ def test_summarize_clocks_keeps_only_the_timed_window():
 
 def test_launch_count_per_path():
     import synth
-    assert bench.launches_per_step(synth.workload(5)) == 6   # fp8 MLA: + query split
-    assert bench.launches_per_step(synth.workload(4)) == 5
-    assert bench.launches_per_step(synth.workload(3)) == 5
+    # shard map, append, plan, decode (with the merge inside); fp8 MLA adds the query split
+    assert bench.launches_per_step(synth.workload(5)) == 5
+    assert bench.launches_per_step(synth.workload(4)) == 4
+    assert bench.launches_per_step(synth.workload(3)) == 4
+
+
+def test_band_latency_summary():
+    """Requests fall in the bands by length; percentiles and the band's rate come from
+    the per-request completion times."""
+    import numpy as np
+    L = np.array([1_000, 31_999, 32_000, 100_000, 250_000, 250_001])
+    fin = np.array([0.5, 1.0, 1.5, 2.0, 4.0, 3.0])
+    d = bench.band_latency(L, fin, 4.2, 580)
+    assert set(d) == {"<32k", "32-64k", "64-128k", "200k+", "batch_decode_ms"}
+    assert d["<32k"]["requests"] == 2 and d["<32k"]["tokens"] == 32_999
+    assert d["<32k"]["done_ms_max"] == 1.0 and d["<32k"]["done_ms_p50"] == 0.75
+    assert d["200k+"]["done_ms_max"] == 4.0
+    assert d["32-64k"]["kv_gbs_by_band_done"] == round(32_000 * 580 / 1.5e-3 / 1e9, 1)
+    assert d["batch_decode_ms"] == 4.2
 
 
 def test_traffic_digest_is_per_kernel(tmp_path, monkeypatch):

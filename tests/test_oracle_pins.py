@@ -496,3 +496,24 @@ def test_quantize_rows_matches_single_rows():
     for i in range(40):
         c1, s1 = oracle.quantize_row_e4m3(rows[i])
         assert np.array_equal(codes[i], c1) and sc[i] == np.float32(s1)
+
+
+def test_multi_query_synth_source_equals_array_source():
+    """decode_multi_synth reads the generator as decode_multi_arrays reads the
+    same rows materialised; with one query token it is decode_synth."""
+    seed, B, QL, Hq, Hkv, D = 17, 2, 3, 4, 2, 8
+    L = np.array([5, 70])
+    q = synth.bf16_bits_to_f64(synth.q_bf16(seed, B, QL * Hq, D)).reshape(B, QL, Hq, D)
+    K = np.zeros((B, 70, Hkv, D))
+    V = np.zeros((B, 70, Hkv, D))
+    for b in range(B):
+        K[b] = synth.bf16_bits_to_f64(synth.kv_rows_bf16(seed, synth.T_K, b, np.arange(70), Hkv, D))
+        V[b] = synth.bf16_bits_to_f64(synth.kv_rows_bf16(seed, synth.T_V, b, np.arange(70), Hkv, D))
+    for N, I, shard in ((1, 1, -1), (3, 2, 1)):
+        Oa, la = oracle.decode_multi_arrays("gqa", q, K, V, L, 0.3, N=N, I=I, shard=shard)
+        Os, ls = oracle.decode_multi_synth("gqa", "bf16", seed, q, L, 0.3, Hkv, D, D, N=N, I=I, shard=shard)
+        assert np.array_equal(Oa, Os) and np.array_equal(la, ls)
+    q1 = synth.bf16_bits_to_f64(synth.q_bf16(seed, B, Hq, D))
+    O1, l1 = oracle.decode_synth("gqa", "bf16", seed, q1, L, 0.3, Hkv, D, D)
+    Om, lm = oracle.decode_multi_synth("gqa", "bf16", seed, q1[:, None], L, 0.3, Hkv, D, D)
+    assert np.array_equal(O1, Om[:, 0]) and np.array_equal(l1, lm[:, 0])
