@@ -17,11 +17,12 @@
  *    cp_kv_cache_interleave_size sets how many consecutive positions go to
  *    one shard before moving to the next.
  *
- * This library runs all N shards on ONE GPU: shard n's pages live in the same
+ * The library runs all N shards on ONE GPU: shard n's pages live in the same
  * page pool as the other shards' pages (disjoint page ids), decode_partial
  * computes every shard's partial in one launch, and dcp_merge performs the
  * LSE-weighted sum that the all-gather + reduce-scatter would perform across
- * GPUs.
+ * GPUs (dcp_decode_merged does both in one launch sequence).  The *_rank calls
+ * serve one rank of an N-GPU group instead, whose cache holds only its shard.
  *
  * Conventions for every call:
  *  - Every pointer argument is DEVICE memory owned by the caller, unless the
@@ -201,10 +202,11 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
 
 /*
  * dcp_decode_workspace_size_ex -- bytes of device workspace that
- * dcp_decode_partial_multi (merged = 0) or dcp_decode_merged (merged != 0)
- * needs for this cache, batch and query length on the CURRENT device (host
- * function; no GPU work).  Returns 0 for an invalid descriptor or a shape no
- * kernel of this build covers.
+ * dcp_decode_partial_multi (merged = 0), dcp_decode_merged (merged = 1) or
+ * dcp_decode_rank (merged = 2) needs for this cache, batch and query length on
+ * the CURRENT device (host function; no GPU work).  Returns 0 for an invalid
+ * descriptor, another value of merged, or a shape no kernel of this build
+ * covers.
  */
 size_t dcp_decode_workspace_size_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_len, int32_t merged);
 
@@ -263,6 +265,56 @@ dcp_status dcp_decode_partial_multi(const dcp_cache_desc* cache, int32_t B, int3
 dcp_status dcp_decode_merged(const dcp_cache_desc* cache, int32_t B, int32_t q_len, const void* q,
                              const int32_t* seq_lens, float* out, float* lse_out, int64_t* finish_ns, void* ws,
                              size_t ws_bytes, void* stream);
+
+/*
+ * Several GPUs: the cache of ONE rank of an N-GPU group.
+ * Passage: blog section 4 (each GPU keeps the KV of the positions it owns) and
+ * section 4.1 (each GPU attends its local slice; the partial outputs and LSEs
+ * are then combined by an all-gather and a reduce-scatter across the group).
+ * For these calls the descriptor is that rank's: n_shards = N (the group size),
+ * the pools hold only this rank's pages, and block_tables is int32
+ * [1][batch][max_local_pages]: this rank's local pages of each request.
+ */
+
+/*
+ * dcp_kv_append_rank -- dcp_kv_append on rank `rank`'s cache: every rank may
+ * be given every new token; it stores the ones it owns ((p / I) mod N == rank)
+ * and skips the others without an error.
+ */
+dcp_status dcp_kv_append_rank(const dcp_cache_desc* cache, int32_t rank, int64_t n_tok, const int32_t* req,
+                              const int32_t* pos, const void* k_new, const void* v_new, void* stream);
+
+/*
+ * dcp_decode_rank -- this rank's partial attention: every query token of every
+ * request against the positions rank `rank` owns (0 <= rank < n_shards).
+ *  q_len, q, seq_lens   as dcp_decode_partial_multi (q_len = 1: one token).
+ *  o          fp32 [B][q_len][hq][dv]: the normalised partial output, 0 where
+ *             the rank owns no attended position.
+ *  lse        fp32 [B][q_len][hq]: its natural-log LSE, -inf where none.
+ *  ws, ws_bytes  at least dcp_decode_workspace_size_ex(cache, B, q_len, 2).
+ * Next: all-gather lse across the group, dcp_lse_rescale, reduce-scatter.
+ * Errors as dcp_decode_partial.
+ */
+dcp_status dcp_decode_rank(const dcp_cache_desc* cache, int32_t rank, int32_t B, int32_t q_len, const void* q,
+                           const int32_t* seq_lens, float* o, float* lse, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * dcp_lse_rescale -- the local step between the all-gather of the LSEs and the
+ * reduce-scatter of the outputs (blog section 4.1: the LSE values reweight the
+ * partials, the reduce-scatter sums them).
+ *  lse_all    fp32 [N][B][H]: every rank's lse (the all-gathered tensor).
+ *  o          fp32 [B][H][Dv]: this rank's partial (dcp_decode_rank's o, with
+ *             H = q_len * hq rows).
+ *  o_rs       fp32 [N][B][H/N][Dv], output: exp(lse_rank - LSE) * o, laid out
+ *             so that block n holds the rows rank n keeps after the
+ *             reduce-scatter (a sum over ranks).  H must be a multiple of N.
+ *  lse_out    fp32 [B][H] or NULL: LSE = M + ln sum_n exp(lse_n - M),
+ *             M = max_n lse_n (-inf when every rank has -inf).
+ * Errors: DCP_ERR_INVALID_ARG for sizes out of range, rank outside [0, N),
+ * H % N != 0 or NULL pointers; DCP_ERR_MISALIGNED for o / o_rs.
+ */
+dcp_status dcp_lse_rescale(int32_t N, int32_t rank, int32_t B, int32_t H, int32_t Dv, const float* lse_all,
+                           const float* o, float* o_rs, float* lse_out, void* stream);
 
 /*
  * DCP_STATIC_SCRATCH_BYTES -- size of the decode scratch built into the

@@ -11,7 +11,9 @@ Entry points (same names as ``include/dcp.h``): ``dcp_shard_counts``,
 ``dcp_shard_map``, ``dcp_kv_append``, ``dcp_decode_workspace_size``,
 ``dcp_decode_workspace_size_ex``, ``dcp_decode_partial``,
 ``dcp_decode_partial_multi``, ``dcp_decode_merged``,
-``dcp_decode_partial_noalloc``, ``dcp_merge``, ``dcp_get_device_status``.
+``dcp_decode_partial_noalloc``, ``dcp_merge``, ``dcp_get_device_status``, and for
+one rank of a multi-GPU group ``dcp_kv_append_rank``, ``dcp_decode_rank``,
+``dcp_lse_rescale`` (the collectives around them are in ``parallel.py``).
 """
 from __future__ import annotations
 
@@ -38,7 +40,7 @@ DCP_FP8_E4M3 = 1
 EXPORTED = ("dcp_status_string", "dcp_shard_counts", "dcp_shard_map", "dcp_kv_append",
             "dcp_decode_workspace_size", "dcp_decode_workspace_size_ex", "dcp_decode_partial",
             "dcp_decode_partial_multi", "dcp_decode_merged", "dcp_decode_partial_noalloc", "dcp_merge",
-            "dcp_get_device_status")
+            "dcp_get_device_status", "dcp_kv_append_rank", "dcp_decode_rank", "dcp_lse_rescale")
 
 
 class DcpError(RuntimeError):
@@ -85,12 +87,15 @@ def lib() -> ctypes.CDLL:
         L.dcp_decode_workspace_size_ex.restype = ctypes.c_size_t
         L.dcp_decode_partial_multi.argtypes = [D, i32, i32, P, P, P, P, P, ctypes.c_size_t, P]
         L.dcp_decode_merged.argtypes = [D, i32, i32, P, P, P, P, P, P, ctypes.c_size_t, P]
+        L.dcp_kv_append_rank.argtypes = [D, i32, i64, P, P, P, P, P]
+        L.dcp_decode_rank.argtypes = [D, i32, i32, i32, P, P, P, P, P, ctypes.c_size_t, P]
+        L.dcp_lse_rescale.argtypes = [i32, i32, i32, i32, i32, P, P, P, P, P]
         L.dcp_decode_partial_noalloc.argtypes = [D, i32, P, P, P, P, P]
         L.dcp_merge.argtypes = [i32, i32, i32, i32, P, P, P, P, P]
         L.dcp_get_device_status.argtypes = [ctypes.POINTER(i32), P]
         for name in ("dcp_shard_counts", "dcp_shard_map", "dcp_kv_append", "dcp_decode_partial",
                      "dcp_decode_partial_multi", "dcp_decode_merged", "dcp_decode_partial_noalloc", "dcp_merge",
-                     "dcp_get_device_status"):
+                     "dcp_get_device_status", "dcp_kv_append_rank", "dcp_decode_rank", "dcp_lse_rescale"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -172,6 +177,26 @@ def dcp_decode_merged(desc: CacheDesc, q, seq_lens, out, lse_out, ws, finish_ns=
     _check(lib().dcp_decode_merged(ctypes.byref(desc), q.shape[0], q_len, _ptr(q), _ptr(seq_lens), _ptr(out),
                                    _ptr(lse_out), _ptr(finish_ns), _ptr(ws), ws.numel() * ws.element_size(),
                                    _stream(stream)), "dcp_decode_merged")
+
+
+def dcp_kv_append_rank(desc: CacheDesc, rank: int, req, pos, k_new, v_new=None, stream=None) -> None:
+    _check(lib().dcp_kv_append_rank(ctypes.byref(desc), rank, pos.numel(), _ptr(req), _ptr(pos), _ptr(k_new),
+                                    _ptr(v_new), _stream(stream)), "dcp_kv_append_rank")
+
+
+def dcp_decode_rank(desc: CacheDesc, rank: int, q, seq_lens, o, lse, ws, stream=None) -> None:
+    """Rank `rank`'s partial: q bf16 [B][hq][dk] or [B][q_len][hq][dk] -> o, lse with q's leading dims."""
+    q_len = 1 if q.dim() == 3 else q.shape[1]
+    _check(lib().dcp_decode_rank(ctypes.byref(desc), rank, q.shape[0], q_len, _ptr(q), _ptr(seq_lens), _ptr(o),
+                                 _ptr(lse), _ptr(ws), ws.numel() * ws.element_size(), _stream(stream)),
+           "dcp_decode_rank")
+
+
+def dcp_lse_rescale(lse_all, rank: int, o, o_rs, lse_out=None, stream=None) -> None:
+    """lse_all [N][B][H], o [B][H][Dv] -> o_rs [N][B][H/N][Dv] (reduce-scatter layout), lse_out [B][H]."""
+    N, B, H = lse_all.shape
+    _check(lib().dcp_lse_rescale(N, rank, B, H, o.shape[-1], _ptr(lse_all), _ptr(o), _ptr(o_rs), _ptr(lse_out),
+                                 _stream(stream)), "dcp_lse_rescale")
 
 
 # size of the library's built-in decode scratch (DCP_STATIC_SCRATCH_BYTES in dcp.h)

@@ -148,9 +148,12 @@ void add_query_split(const dcp_cache_desc* c, int B, Plan* p) {
     p->lay.total = align256(p->off_qinv + (size_t)B * 64 * sizeof(float));
 }
 
-// Split slots: per-shard groups only split shards longer than one chunk, which
-// gives at most 2 * target + 2 slots; a merged group takes one slot per unit.
-int64_t split_bound(int64_t target, int64_t max_units, int merged) { return merged ? max_units : 2 * target + 2; }
+// Split slots: chunk slots only for shards longer than one chunk, which gives
+// at most 2 * target + 2 of them; merged outputs add one slot per shard with
+// tokens (at most N * B).
+int64_t split_bound(int64_t target, int64_t n_shard_slots, int merged) {
+    return 2 * target + 2 + (merged ? n_shard_slots : 0);
+}
 
 // The plan of a decode of B requests with q_len query tokens each (q_len * hq
 // query rows); merged != 0 gathers every shard of a request into one output
@@ -162,7 +165,7 @@ bool make_plan(const dcp_cache_desc* c, int B, int q_len, int merged, int num_sm
     if (q_len > 1 && p->g.path != DecodePath::GqaMma && p->g.path != DecodePath::MlaUmma) return false;
     const int64_t target = (int64_t)p->g.units_per_cta * p->g.ctas;
     const int64_t max_units = (int64_t)c->n_shards * B + target + 1;
-    const int64_t max_split = split_bound(target, max_units, merged);
+    const int64_t max_split = split_bound(target, (int64_t)c->n_shards * B, merged);
     if (max_units > (1 << 30)) return false;
     p->lay = ws_layout(c->n_shards, B, rows, c->dv, (int)max_units, (int)max_split);
     p->q_len = q_len;
@@ -210,14 +213,17 @@ bool make_plan_within(const dcp_cache_desc* c, int B, int num_sms, size_t cap, P
 
 // The launch sequence of the decode (plan kernel, decode kernel) on a workspace
 // `w` laid out by `p`.
+// rank >= 0: the cache holds only shard `rank`'s block tables, and only that
+// shard is decoded (merged plans only).
 dcp_status decode_on(const dcp_cache_desc* cache, int32_t B, const void* q, const int32_t* seq_lens,
                      float* o_partial, float* lse, uint8_t* w, const Plan& p, int* status, cudaStream_t s,
-                     int64_t* finish_ns = nullptr) {
+                     int64_t* finish_ns = nullptr, int rank = -1) {
     const int64_t target = (int64_t)p.g.units_per_cta * p.g.ctas;
     const int rows = p.q_len * cache->hq;
-    cudaError_t e = launch_plan(seq_lens, B, cache->n_shards, cache->interleave, p.q_len, p.merged, p.g.granule,
-                                p.g.min_chunk, (int)target, p.g.n_hb, w, p.lay.max_units, p.lay.max_split, rows,
-                                cache->dv, finish_ns, status, s);
+    const int shard_lo = rank >= 0 ? rank : 0, shard_hi = rank >= 0 ? rank + 1 : cache->n_shards;
+    cudaError_t e = launch_plan(seq_lens, B, cache->n_shards, cache->interleave, p.q_len, p.merged, shard_lo,
+                                shard_hi, p.g.granule, p.g.min_chunk, (int)target, p.g.n_hb, w, p.lay.max_units,
+                                p.lay.max_split, rows, cache->dv, finish_ns, status, s);
     if (e != cudaSuccess) return DCP_ERR_CUDA;
     DecodeArgs a;
     a.k_pages = static_cast<const uint8_t*>(cache->k_pages);
@@ -250,6 +256,7 @@ dcp_status decode_on(const dcp_cache_desc* cache, int32_t B, const void* q, cons
     a.status = status;
     a.q_len = p.q_len;
     a.finish_ns = finish_ns;
+    a.bt_shard0 = rank >= 0 ? rank : 0;
     e = launch_decode(p.g, a, s);
     if (e == cudaErrorNotSupported) return DCP_ERR_UNSUPPORTED;
     return cuda_err(e);
@@ -370,8 +377,8 @@ dcp_status dcp_shard_map(const dcp_cache_desc* cache, int64_t n_pos, const int32
                                      rank_out, local_out, slot_out, status, (cudaStream_t)stream));
 }
 
-dcp_status dcp_kv_append(const dcp_cache_desc* cache, int64_t n_tok, const int32_t* req, const int32_t* pos,
-                         const void* k_new, const void* v_new, void* stream) {
+static dcp_status kv_append(const dcp_cache_desc* cache, int32_t only_shard, int64_t n_tok, const int32_t* req,
+                            const int32_t* pos, const void* k_new, const void* v_new, void* stream) {
     dcp_status st = check_desc(cache, true);
     if (st != DCP_OK) return st;
     if (n_tok < 0) return DCP_ERR_INVALID_ARG;
@@ -403,7 +410,19 @@ dcp_status dcp_kv_append(const dcp_cache_desc* cache, int64_t n_tok, const int32
     a.kv_scales = cache->kv_scales;
     a.block_tables = cache->block_tables;
     a.status = status;
+    a.only_shard = only_shard;
     return cuda_err(launch_append(a, (cudaStream_t)stream));
+}
+
+dcp_status dcp_kv_append(const dcp_cache_desc* cache, int64_t n_tok, const int32_t* req, const int32_t* pos,
+                         const void* k_new, const void* v_new, void* stream) {
+    return kv_append(cache, -1, n_tok, req, pos, k_new, v_new, stream);
+}
+
+dcp_status dcp_kv_append_rank(const dcp_cache_desc* cache, int32_t rank, int64_t n_tok, const int32_t* req,
+                              const int32_t* pos, const void* k_new, const void* v_new, void* stream) {
+    if (!cache || rank < 0 || rank >= cache->n_shards) return DCP_ERR_INVALID_ARG;
+    return kv_append(cache, rank, n_tok, req, pos, k_new, v_new, stream);
 }
 
 size_t dcp_decode_workspace_size(const dcp_cache_desc* cache, int32_t B) {
@@ -420,7 +439,8 @@ size_t dcp_decode_workspace_size_ex(const dcp_cache_desc* cache, int32_t B, int3
     int num_sms = 0;
     if (device_info(nullptr, &num_sms) != DCP_OK) return 0;
     Plan p;
-    if (!make_plan(cache, B, q_len, merged ? 1 : 0, num_sms, &p)) return 0;
+    // mode 2 (one rank's shard) plans like the merged output over fewer shards
+    if (merged < 0 || merged > 2 || !make_plan(cache, B, q_len, merged ? 1 : 0, num_sms, &p)) return 0;
     return p.lay.total;
 }
 
@@ -440,12 +460,14 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
     return decode_on(cache, B, q, seq_lens, o_partial, lse, static_cast<uint8_t*>(ws), p, status, (cudaStream_t)stream);
 }
 
-// Shared checks and launch of the two decode calls that take a query length.
+// Shared checks and launch of the decode calls that take a query length
+// (rank >= 0: only that shard, from a cache holding only its tables).
 static dcp_status decode_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_len, int merged, const void* q,
                             const int32_t* seq_lens, float* out, float* lse, int64_t* finish_ns, void* ws,
-                            size_t ws_bytes, void* stream) {
+                            size_t ws_bytes, void* stream, int rank = -1) {
     dcp_status st = check_desc(cache, true);
     if (st != DCP_OK) return st;
+    if (rank >= cache->n_shards) return DCP_ERR_INVALID_ARG;
     if (B != cache->batch || q_len < 1 || !q || !seq_lens || !out || !lse || !ws) return DCP_ERR_INVALID_ARG;
     if (q_len > kMaxQueryLen) return DCP_ERR_UNSUPPORTED;
     if (!aligned16(q) || !aligned16(out) || !aligned16(lse) || !aligned16(ws) || (finish_ns && !aligned16(finish_ns)))
@@ -458,7 +480,7 @@ static dcp_status decode_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_le
     if (!make_plan(cache, B, q_len, merged, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
     if (ws_bytes < p.lay.total) return DCP_ERR_WORKSPACE_TOO_SMALL;
     return decode_on(cache, B, q, seq_lens, out, lse, static_cast<uint8_t*>(ws), p, status, (cudaStream_t)stream,
-                     finish_ns);
+                     finish_ns, rank);
 }
 
 dcp_status dcp_decode_partial_multi(const dcp_cache_desc* cache, int32_t B, int32_t q_len, const void* q,
@@ -471,6 +493,12 @@ dcp_status dcp_decode_merged(const dcp_cache_desc* cache, int32_t B, int32_t q_l
                              const int32_t* seq_lens, float* out, float* lse_out, int64_t* finish_ns, void* ws,
                              size_t ws_bytes, void* stream) {
     return decode_ex(cache, B, q_len, 1, q, seq_lens, out, lse_out, finish_ns, ws, ws_bytes, stream);
+}
+
+dcp_status dcp_decode_rank(const dcp_cache_desc* cache, int32_t rank, int32_t B, int32_t q_len, const void* q,
+                           const int32_t* seq_lens, float* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
+    if (!cache || rank < 0) return DCP_ERR_INVALID_ARG;
+    return decode_ex(cache, B, q_len, 1, q, seq_lens, o, lse, nullptr, ws, ws_bytes, stream, rank);
 }
 
 // No workspace argument and no allocation: for callers that cannot allocate
@@ -502,6 +530,14 @@ dcp_status dcp_merge(int32_t N, int32_t B, int32_t H, int32_t Dv, const float* o
     if (N < 1 || B < 1 || H < 1 || Dv < 4 || Dv % 4 || !o_partial || !lse || !out) return DCP_ERR_INVALID_ARG;
     if (!aligned16(o_partial) || !aligned16(out)) return DCP_ERR_MISALIGNED;
     return cuda_err(launch_merge(N, B, H, Dv, o_partial, lse, out, lse_out, (cudaStream_t)stream));
+}
+
+dcp_status dcp_lse_rescale(int32_t N, int32_t rank, int32_t B, int32_t H, int32_t Dv, const float* lse_all,
+                           const float* o, float* o_rs, float* lse_out, void* stream) {
+    if (N < 1 || rank < 0 || rank >= N || B < 1 || H < 1 || H % N || Dv < 4 || Dv % 4 || !lse_all || !o || !o_rs)
+        return DCP_ERR_INVALID_ARG;
+    if (!aligned16(o) || !aligned16(o_rs)) return DCP_ERR_MISALIGNED;
+    return cuda_err(launch_lse_rescale(N, rank, B, H, Dv, lse_all, o, o_rs, lse_out, (cudaStream_t)stream));
 }
 
 dcp_status dcp_get_device_status(int32_t* status_out, void* stream) {

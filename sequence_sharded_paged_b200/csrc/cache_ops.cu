@@ -53,12 +53,17 @@ __global__ void shard_map_kernel(int64_t n_pos, const int32_t* __restrict__ pos,
     }
 }
 
-// Resolve (req, pos) -> physical page and in-page offset; -1 page when invalid.
+// Resolve (req, pos) -> physical page and in-page offset; -1 page when invalid,
+// -2 when another rank owns the position (rank-local cache).
 __device__ __forceinline__ int append_target(const AppendArgs& a, int64_t i, int* off) {
     int64_t p = a.pos[i];
     int b = a.req ? a.req[i] : (int)i;
     if (p < 0 || b < 0 || b >= a.batch) return -1;
     int r = owner_of(p, a.n_shards, a.interleave);
+    if (a.only_shard >= 0) {
+        if (r != a.only_shard) return -2;
+        r = 0;  // the rank's tables are row 0
+    }
     int64_t l = local_of(p, a.n_shards, a.interleave);
     int64_t j = l / a.page_size;
     if (j >= a.max_local_pages) return -1;
@@ -78,7 +83,7 @@ __global__ void append_gqa_kernel(AppendArgs a) {
     int off = 0;
     int pg = append_target(a, i, &off);
     if (pg < 0) {
-        if (lane == 0) record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
+        if (pg == -1 && lane == 0) record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
         return;
     }
     const int P = a.page_size;
@@ -102,7 +107,7 @@ __global__ void append_mla_bf16_kernel(AppendArgs a) {
     int off = 0;
     int pg = append_target(a, i, &off);
     if (pg < 0) {
-        if (lane == 0) record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
+        if (pg == -1 && lane == 0) record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
         return;
     }
     const uint4* src = reinterpret_cast<const uint4*>(a.k_new + i * a.dk * 2);
@@ -119,7 +124,7 @@ __global__ void append_mla_fp8_kernel(AppendArgs a) {
     int off = 0;
     int pg = append_target(a, i, &off);
     if (pg < 0) {
-        if (lane == 0) record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
+        if (pg == -1 && lane == 0) record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
         return;
     }
     // 576 bf16 = 72 chunks of 8; lane owns chunks lane, lane+32, lane+64 (< 72)

@@ -159,17 +159,20 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // work units produced by the planner
 // ---------------------------------------------------------------------------
 struct Unit {
-    int32_t n;          // shard
-    int32_t b;          // request
-    int32_t t0, t1;     // local token range [t0, t1) of shard n of request b
-    int32_t slot;       // split-partial slot of this unit, -1 when its group has one unit
-    int32_t n_chunks;   // units of this unit's output group
-    int32_t slot_base;  // first split slot of the group
-    int32_t grp;        // output group: row block grp of the outputs (n*B + b for per-shard
-                        // partials, b for the merged output); the group's last unit to finish
-                        // LSE-merges its units' split partials there
+    int32_t n;           // shard
+    int32_t b;           // request
+    int32_t t0, t1;      // local token range [t0, t1) of shard n of request b
+    int32_t slot;        // chunk slot of this unit, -1 when its shard is one unit
+    int32_t n_chunks;    // units (chunks) of this unit's shard
+    int32_t slot_base;   // first chunk slot of the shard
+    int32_t grp;         // output row block: n*B + b (per-shard partials) or b (merged output)
+    int32_t sslot;       // merged output: slot of this shard's partial in its request's merge,
+                         // -1 when the request has a single shard with tokens (or per-shard outputs)
+    int32_t n_sh;        // merged output: shards with tokens in the request (else 1)
+    int32_t sslot_base;  // merged output: first shard slot of the request
+    int32_t pad;
 };
-static_assert(sizeof(Unit) == 32, "Unit layout");
+static_assert(sizeof(Unit) == 48, "Unit layout");
 
 struct PlanHeader {
     int32_t num_units;
@@ -200,8 +203,10 @@ constexpr int kStageLast = 2;
 constexpr int kStageValid = 4;
 
 // Workspace layout (all offsets 256-byte aligned):
-//   PlanHeader | Unit[max_units] | int32 done[N*B] | int32 shard_k[N*B] |
+//   PlanHeader | Unit[max_units] | int32 done[(N+1)*B*hq] | int32 shard_k[N*B] |
 //   int32 slot_base[N*B] | float split_o[max_split][hq][dv] | float split_lse[max_split][hq]
+// done: counters per (shard, request, head block) for the chunks of a shard,
+// then per (request, head block) for the shards of a request (merged output).
 struct WsLayout {
     size_t off_units, off_done, off_k, off_base, off_split_o, off_split_lse, total;
     int32_t max_units, max_split;
@@ -214,8 +219,8 @@ __host__ inline WsLayout ws_layout(int N, int B, int hq, int dv, int max_units, 
     size_t o = align256(sizeof(PlanHeader));
     w.off_units = o;
     o = align256(o + sizeof(Unit) * (size_t)max_units);
-    w.off_done = o;  // one counter per (shard, request, head block); head blocks <= hq
-    o = align256(o + sizeof(int32_t) * (size_t)N * B * hq);
+    w.off_done = o;  // counters per (shard or request, head block); head blocks <= hq
+    o = align256(o + sizeof(int32_t) * (size_t)(N + 1) * B * hq);
     w.off_k = o;
     o = align256(o + sizeof(int32_t) * (size_t)N * B);
     w.off_base = o;
@@ -259,6 +264,10 @@ struct DecodeArgs {
     // r = j * (hq / q_len) + head belongs to query token j
     int32_t q_len;
     int64_t* finish_ns;  // per output group: ns from the planner's start to its final output (or null)
+    // first shard whose block tables are present: 0 when block_tables holds every
+    // shard ([N][B][max_local_pages]); r when it holds only shard r's ([1][B][..]),
+    // the cache of rank r of a multi-GPU group
+    int32_t bt_shard0;
 };
 
 // Local tokens [0, limit) of shard u.n that query token j attends: the positions
@@ -287,7 +296,7 @@ __device__ __forceinline__ void discard_l2_line(const void* p) {
 // Fetch the physical page of local page j of (n, b); -1 when invalid.
 __device__ __forceinline__ int page_of(const DecodeArgs& a, int n, int b, int j) {
     if (j >= a.max_local_pages) return -1;
-    int pg = __ldg(a.block_tables + ((int64_t)n * a.batch + b) * a.max_local_pages + j);
+    int pg = __ldg(a.block_tables + ((int64_t)(n - a.bt_shard0) * a.batch + b) * a.max_local_pages + j);
     return (pg >= 0 && pg < a.num_pages) ? pg : -1;
 }
 

@@ -17,9 +17,12 @@
 //
 // Structure: persistent grid, one work unit (shard, request, chunk) per CTA
 // iteration, all KV heads in the CTA.  Warp NCW (producer) issues TMA tiled
-// loads of 16-token stages -- for every KV head and 64-column half a
-// [16 tokens][64] box of K and of V with 128-byte swizzle -- into a ring of
-// shared-memory stages (mbarrier complete_tx).  Consumer warp w owns KV head
+// loads of 16-token stages into a ring of shared-memory stages (mbarrier
+// complete_tx): one 4-D box for K and one for V, which view the pool as
+// [page * Hkv + head][64-column half][token][64 columns] and land as
+// [head][half][16 tokens][128 B] with 128-byte swizzle (the copy engine's
+// cost is per copy, so a stage is two copies rather than one per head and
+// half).  Consumer warp w owns KV head
 // w % Hkv and every (NCW/Hkv)-th stage: S = Q K^T (ldmatrix), online softmax
 // in registers (quad shuffles), O += P V (ldmatrix.trans).  At the end of the
 // unit the warps' states are merged through shared memory.
@@ -70,10 +73,12 @@ __device__ __forceinline__ uint32_t swz(int r, int c) {
     return (uint32_t)(r * 128 + ((((c >> 3) ^ (r & 7)) & 7) << 4) + ((c & 7) << 1));
 }
 
+// tmK / tmV: 4-D maps (one copy per stage each) when map4 != 0, else 2-D maps of
+// [16 tokens][64 columns] boxes (one copy per head and half).
 template <int D, int NCW>
 __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid_constant__ CUtensorMap tmK,
                                                                  const __grid_constant__ CUtensorMap tmV,
-                                                                 DecodeArgs a, int stages) {
+                                                                 DecodeArgs a, int stages, int map4) {
     constexpr int HALVES = D / 64;
     constexpr int NT = 32 * NCW;
     extern __shared__ __align__(1024) uint8_t smem_raw[];
@@ -143,14 +148,20 @@ __global__ void __launch_bounds__(32 * (NCW + 1), 1) gqa_mma_kernel(const __grid
                         smeta[stage] = StageMeta{ui, t, flags | kStageValid, k};
                         mbar_arrive_expect_tx(full + stage, stage_bytes);
                         uint8_t* st = ring + (size_t)stage * stage_bytes;
-                        for (int g = 0; g < hkv; g++) {
-                            const int row = (pg * hkv + g) * P + sub * kTok;
+                        if (map4) {
+                            tma_load_4d(st, &tmK, 0, sub * kTok, 0, pg * hkv, full + stage, pol);
+                            tma_load_4d(st + (size_t)hkv * HALVES * kBoxBytes, &tmV, 0, sub * kTok, 0, pg * hkv,
+                                        full + stage, pol);
+                        } else {
+                            for (int g = 0; g < hkv; g++) {
+                                const int row = (pg * hkv + g) * P + sub * kTok;
 #pragma unroll
-                            for (int h = 0; h < HALVES; h++) {
-                                tma_load_2d(st + ((size_t)(g * HALVES + h)) * kBoxBytes, &tmK, h * 64, row,
-                                            full + stage, pol);
-                                tma_load_2d(st + ((size_t)((hkv + g) * HALVES + h)) * kBoxBytes, &tmV, h * 64, row,
-                                            full + stage, pol);
+                                for (int h = 0; h < HALVES; h++) {
+                                    tma_load_2d(st + ((size_t)(g * HALVES + h)) * kBoxBytes, &tmK, h * 64, row,
+                                                full + stage, pol);
+                                    tma_load_2d(st + ((size_t)((hkv + g) * HALVES + h)) * kBoxBytes, &tmV, h * 64,
+                                                row, full + stage, pol);
+                                }
                             }
                         }
                     } else {
@@ -416,18 +427,29 @@ int gqa_mma_stages(int hq, int hkv) {
 template <int D, int NCW>
 cudaError_t run(const DecodeGeometry& geo, const DecodeArgs& a, cudaStream_t s) {
     CUtensorMap tk, tv;
-    const uint64_t rows = (uint64_t)a.num_pages * a.hkv * a.page_size;
-    if (!make_tmap_2d(&tk, a.k_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, rows, (uint64_t)D * 2, 64, kTok,
-                      CU_TENSOR_MAP_SWIZZLE_128B) ||
-        !make_tmap_2d(&tv, a.v_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, rows, (uint64_t)D * 2, 64, kTok,
-                      CU_TENSOR_MAP_SWIZZLE_128B))
-        return cudaErrorInvalidValue;
+    // [page * Hkv + head][half][token][64 columns] view of each pool; the box is a whole
+    // stage: 64 columns x 16 tokens x every half x every head
+    const uint64_t dims[4] = {64, (uint64_t)a.page_size, (uint64_t)(D / 64), (uint64_t)a.num_pages * a.hkv};
+    const uint64_t strides[3] = {(uint64_t)D * 2, 128, (uint64_t)a.page_size * D * 2};
+    const uint32_t box[4] = {64, (uint32_t)kTok, (uint32_t)(D / 64), (uint32_t)a.hkv};
+    int map4 = make_tmap_4d(&tk, a.k_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dims, strides, box,
+                            CU_TENSOR_MAP_SWIZZLE_128B) &&
+               make_tmap_4d(&tv, a.v_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, dims, strides, box,
+                            CU_TENSOR_MAP_SWIZZLE_128B);
+    if (!map4) {
+        const uint64_t rows = (uint64_t)a.num_pages * a.hkv * a.page_size;
+        if (!make_tmap_2d(&tk, a.k_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, rows, (uint64_t)D * 2, 64, kTok,
+                          CU_TENSOR_MAP_SWIZZLE_128B) ||
+            !make_tmap_2d(&tv, a.v_pages, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, D, rows, (uint64_t)D * 2, 64, kTok,
+                          CU_TENSOR_MAP_SWIZZLE_128B))
+            return cudaErrorInvalidValue;
+    }
     const int stages = gqa_mma_stages<D, NCW>(a.hq, a.hkv);
     const size_t smem = gqa_mma_smem<D, NCW>(a.hq, a.hkv, stages);
     cudaError_t e = cudaFuncSetAttribute(gqa_mma_kernel<D, NCW>, cudaFuncAttributeMaxDynamicSharedMemorySize,
                                          (int)smem);
     if (e != cudaSuccess) return e;
-    gqa_mma_kernel<D, NCW><<<geo.ctas, 32 * (NCW + 1), smem, s>>>(tk, tv, a, stages);
+    gqa_mma_kernel<D, NCW><<<geo.ctas, 32 * (NCW + 1), smem, s>>>(tk, tv, a, stages, map4);
     return cudaGetLastError();
 }
 

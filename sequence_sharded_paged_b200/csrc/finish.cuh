@@ -15,102 +15,162 @@ __device__ __forceinline__ void named_barrier_sync(int id, int threads) {
     asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(threads) : "memory");
 }
 
-// Merge the split partials of the units of group u.grp for rows h0..h0+nh-1
-// into o_partial / lse (executed by the NT threads of barrier `bar_id`, tid in
-// [0, NT)):
+// Merge the K partials in split slots [base, base + K) for rows h0..h0+nh-1
+// into dst_o [rows][dv] / dst_lse [rows] (rows indexed from 0), executed by
+// warps w0, w0 + 1, .., w0 + nw - 1 of the caller (one warp per row, lane =
+// tid & 31):
 //   M = max_j lse_j,  O = sum_j exp(lse_j - M) O_j / sum_j exp(lse_j - M),
 //   LSE = M + ln sum_j exp(lse_j - M).
-// The partials are dead afterwards, so their L2 lines are discarded: a merge
-// that runs while they are still in L2 keeps them from ever reaching HBM.
-__device__ inline void merge_split_chunks(const DecodeArgs& a, const Unit& u, int h0, int nh, int tid, int NT,
-                                          int bar_id) {
+// The partials are dead afterwards, so each warp discards the L2 lines it has
+// read: a merge that runs while they are still in L2 keeps them from ever
+// reaching HBM.
+__device__ inline void merge_slots(const DecodeArgs& a, int base, int K, int h0, int nh, float* dst_o,
+                                   float* dst_lse, int w, int nw, int lane) {
+    constexpr int kMaxV = 4;  // float4 per lane and row: dv <= 512
     const int dv = a.dv;
-    const int K = u.n_chunks;
-    const int64_t grp = u.grp;
-    for (int i = tid; i < nh * (dv / 4); i += NT) {
-        const int h = i / (dv / 4), d4 = i - h * (dv / 4);
-        const float* lse_col = a.split_lse + (int64_t)u.slot_base * a.hq + h0 + h;
+    const int nv = dv / 4;
+    for (int h = w; h < nh; h += nw) {
+        const float* lse_col = a.split_lse + (int64_t)base * a.hq + h0 + h;
         float M = -INFINITY;
-        for (int j = 0; j < K; j++) M = fmaxf(M, __ldcg(lse_col + (int64_t)j * a.hq));
-        float4 o = make_float4(0.f, 0.f, 0.f, 0.f);
+        for (int j = lane; j < K; j += 32) M = fmaxf(M, __ldcg(lse_col + (int64_t)j * a.hq));
+#pragma unroll
+        for (int o = 16; o; o >>= 1) M = fmaxf(M, __shfl_xor_sync(0xffffffffu, M, o));
         float wsum = 0.f;
+        if (M != -INFINITY)
+            for (int j = lane; j < K; j += 32) {
+                const float lj = __ldcg(lse_col + (int64_t)j * a.hq);
+                wsum += lj == -INFINITY ? 0.f : expf(lj - M);
+            }
+#pragma unroll
+        for (int o = 16; o; o >>= 1) wsum += __shfl_xor_sync(0xffffffffu, wsum, o);
+        float4 acc[kMaxV];
+#pragma unroll
+        for (int r = 0; r < kMaxV; r++) acc[r] = make_float4(0.f, 0.f, 0.f, 0.f);
         if (M != -INFINITY) {
+#pragma unroll 8
             for (int j = 0; j < K; j++) {
                 const float lj = __ldcg(lse_col + (int64_t)j * a.hq);
-                if (lj == -INFINITY) continue;
-                const float w = expf(lj - M);
-                wsum += w;
-                const float4 x = __ldcg(
-                    reinterpret_cast<const float4*>(a.split_o + ((int64_t)(u.slot_base + j) * a.hq + h0 + h) * dv) + d4);
-                o.x += w * x.x;
-                o.y += w * x.y;
-                o.z += w * x.z;
-                o.w += w * x.w;
+                const float4* src =
+                    reinterpret_cast<const float4*>(a.split_o + ((int64_t)(base + j) * a.hq + h0 + h) * dv);
+                float4 x[kMaxV];
+#pragma unroll
+                for (int r = 0; r < kMaxV; r++)
+                    x[r] = (lane + 32 * r < nv) ? __ldcg(src + lane + 32 * r) : make_float4(0.f, 0.f, 0.f, 0.f);
+                const float wj = lj == -INFINITY ? 0.f : expf(lj - M);
+#pragma unroll
+                for (int r = 0; r < kMaxV; r++) {
+                    acc[r].x = fmaf(wj, x[r].x, acc[r].x);
+                    acc[r].y = fmaf(wj, x[r].y, acc[r].y);
+                    acc[r].z = fmaf(wj, x[r].z, acc[r].z);
+                    acc[r].w = fmaf(wj, x[r].w, acc[r].w);
+                }
             }
-            const float inv = 1.f / wsum;
-            o.x *= inv;
-            o.y *= inv;
-            o.z *= inv;
-            o.w *= inv;
         }
-        reinterpret_cast<float4*>(a.o_partial + (grp * a.hq + h0 + h) * dv)[d4] = o;
-        if (d4 == 0) a.lse[grp * a.hq + h0 + h] = (M == -INFINITY) ? -INFINITY : M + logf(wsum);
-    }
-    // every thread has consumed its loads (their values are stored above)
-    named_barrier_sync(bar_id, NT);
-    const int lines = dv / 32;  // 128-byte lines per row of dv floats
-    const int n_lines = K * nh * lines;
-    for (int i = tid; i < n_lines; i += NT) {
-        const int j = i / (nh * lines), rem = i - j * nh * lines;
-        const int h = rem / lines, l = rem - h * lines;
-        discard_l2_line(a.split_o + ((int64_t)(u.slot_base + j) * a.hq + h0 + h) * dv + l * 32);
+        const float inv = M != -INFINITY ? 1.f / wsum : 0.f;
+        float4* dst = reinterpret_cast<float4*>(dst_o + (int64_t)(h0 + h) * dv);
+#pragma unroll
+        for (int r = 0; r < kMaxV; r++)
+            if (lane + 32 * r < nv)
+                __stcg(dst + lane + 32 * r, make_float4(acc[r].x * inv, acc[r].y * inv, acc[r].z * inv, acc[r].w * inv));
+        if (lane == 0) __stcg(dst_lse + h0 + h, (M == -INFINITY) ? -INFINITY : M + logf(wsum));
+        // every lane has consumed its loads of this row (the values are stored above)
+        __syncwarp();
+        const int lines = dv / 32;  // 128-byte lines per row of dv floats
+        for (int i = lane; i < K * lines; i += 32) {
+            const int j = i / lines, l = i - j * lines;
+            discard_l2_line(a.split_o + ((int64_t)(base + j) * a.hq + h0 + h) * dv + l * 32);
+        }
     }
 }
 
-// Executed by the NT threads of barrier `bar_id` (tid in [0, NT)).
+// Where a unit's own result goes: its chunk slot when its shard is cut into
+// several chunks; otherwise where its shard's result goes (shard_dst).
+// Where a shard's result goes: its slot in the request's merge (merged output
+// over several shards), else the output row block u.grp.
+__device__ __forceinline__ void shard_dst(const DecodeArgs& a, const Unit& u, float** o, float** lse) {
+    if (u.sslot >= 0) {
+        *o = a.split_o + (int64_t)u.sslot * a.hq * a.dv;
+        *lse = a.split_lse + (int64_t)u.sslot * a.hq;
+    } else {
+        *o = a.o_partial + (int64_t)u.grp * a.hq * a.dv;
+        *lse = a.lse + (int64_t)u.grp * a.hq;
+    }
+}
+__device__ __forceinline__ void unit_dst(const DecodeArgs& a, const Unit& u, float** o, float** lse) {
+    if (u.slot >= 0) {
+        *o = a.split_o + (int64_t)u.slot * a.hq * a.dv;
+        *lse = a.split_lse + (int64_t)u.slot * a.hq;
+    } else {
+        shard_dst(a, u, o, lse);
+    }
+}
+// completion counters: the chunks of shard (u.n, u.b), and the shards of request u.b
+__device__ __forceinline__ int32_t* shard_counter(const DecodeArgs& a, const Unit& u, int hb, int n_hb) {
+    return a.done + ((int64_t)u.n * a.batch + u.b) * n_hb + hb;
+}
+__device__ __forceinline__ int32_t* request_counter(const DecodeArgs& a, const Unit& u, int hb, int n_hb) {
+    return a.done + ((int64_t)a.n_shards * a.batch + u.b) * n_hb + hb;
+}
+
+// Executed by the NT threads of barrier `bar_id` (tid in [0, NT), NT a
+// multiple of 32).
 //  sO   [nh][dv] normalised output of this unit for rows h0..h0+nh-1 (smem)
 //  sLse [nh]     natural-log LSE (-inf when the unit saw no token)
-//  hb / n_hb     head block of this unit and head blocks per unit (split counters
-//                are per (group, head block))
-// Records the group's completion time when a.finish_ns is set.
+//  hb / n_hb     head block of this unit and head blocks per unit (counters are
+//                per (shard or request, head block))
+// Stores the unit's result, then merges its shard's chunks when it completes the
+// shard, then the request's shards when that completes the request (merged
+// output), and records the request's completion time when a.finish_ns is set.
 template <int NT>
 __device__ void finish_unit(const DecodeArgs& a, const Unit& u, int hb, int n_hb, int h0, int nh,
                             const float* sO, const float* sLse, int* s_flag, int tid, int bar_id) {
     const int dv = a.dv;
-    const int64_t grp = u.grp;
     const int nvec = nh * dv / 4;
-    if (u.n_chunks == 1) {
-        float4* dst = reinterpret_cast<float4*>(a.o_partial + (grp * a.hq + h0) * dv);
-        const float4* src = reinterpret_cast<const float4*>(sO);
-        for (int i = tid; i < nvec; i += NT) dst[i] = src[i];
-        for (int i = tid; i < nh; i += NT) a.lse[grp * a.hq + h0 + i] = sLse[i];
-        if (a.finish_ns) {
-            named_barrier_sync(bar_id, NT);
-            if (tid == 0) record_finish(a, (int)grp);
-        }
-        return;
-    }
+    float* o_dst;
+    float* l_dst;
+    unit_dst(a, u, &o_dst, &l_dst);
+    const bool counted = u.slot >= 0 || u.sslot >= 0;  // does anything merge this result later?
     {
-        float4* dst = reinterpret_cast<float4*>(a.split_o + ((int64_t)u.slot * a.hq + h0) * dv);
+        float4* dst = reinterpret_cast<float4*>(o_dst + (int64_t)h0 * dv);
         const float4* src = reinterpret_cast<const float4*>(sO);
         for (int i = tid; i < nvec; i += NT) __stcg(dst + i, src[i]);
-        for (int i = tid; i < nh; i += NT) __stcg(a.split_lse + (int64_t)u.slot * a.hq + h0 + i, sLse[i]);
+        for (int i = tid; i < nh; i += NT) __stcg(l_dst + h0 + i, sLse[i]);
     }
-    __threadfence();
-    named_barrier_sync(bar_id, NT);
-    if (tid == 0) {
-        int old = atomicAdd(a.done + grp * n_hb + hb, 1);
-        *s_flag = (old == u.n_chunks - 1) ? 1 : 0;
-    }
-    named_barrier_sync(bar_id, NT);
-    const int last = *(volatile int*)s_flag;
-    named_barrier_sync(bar_id, NT);
-    if (!last) return;
-    __threadfence();
-    merge_split_chunks(a, u, h0, nh, tid, NT, bar_id);
-    if (a.finish_ns) {
+    bool complete = true;  // has this unit completed its shard (and, without a second level, the request)?
+    if (counted) {
+        __threadfence();
         named_barrier_sync(bar_id, NT);
-        if (tid == 0) record_finish(a, (int)grp);
+        // level 1: the chunks of the shard
+        if (u.slot >= 0) {
+            if (tid == 0) *s_flag = (atomicAdd(shard_counter(a, u, hb, n_hb), 1) == u.n_chunks - 1) ? 1 : 0;
+            named_barrier_sync(bar_id, NT);
+            complete = *(volatile int*)s_flag;
+            named_barrier_sync(bar_id, NT);
+            if (complete) {
+                __threadfence();
+                float *so, *sl;
+                shard_dst(a, u, &so, &sl);
+                merge_slots(a, u.slot_base, u.n_chunks, h0, nh, so, sl, tid >> 5, NT >> 5, tid & 31);
+                __threadfence();
+                named_barrier_sync(bar_id, NT);
+            }
+        }
+        // level 2: the shards of the request
+        if (complete && u.sslot >= 0) {
+            if (tid == 0) *s_flag = (atomicAdd(request_counter(a, u, hb, n_hb), 1) == u.n_sh - 1) ? 1 : 0;
+            named_barrier_sync(bar_id, NT);
+            complete = *(volatile int*)s_flag;
+            named_barrier_sync(bar_id, NT);
+            if (complete) {
+                __threadfence();
+                merge_slots(a, u.sslot_base, u.n_sh, h0, nh, a.o_partial + (int64_t)u.grp * a.hq * dv,
+                            a.lse + (int64_t)u.grp * a.hq, tid >> 5, NT >> 5, tid & 31);
+            }
+        }
+    }
+    if (complete && a.finish_ns) {
+        named_barrier_sync(bar_id, NT);
+        if (tid == 0) record_finish(a, u.grp);
     }
 }
 

@@ -24,6 +24,7 @@ struct AppendArgs {
     float* kv_scales;
     const int32_t* block_tables;
     int* status;
+    int32_t only_shard;  // -1: block_tables holds every shard; r: only shard r's, rows of other shards are skipped
 };
 
 cudaError_t launch_shard_counts(int B, const int32_t* seq_lens, int N, int I, int32_t* counts, int* status,
@@ -35,9 +36,10 @@ cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 
 // planner: splits every (shard, request) into chunks of at most chunk_tokens and
 // gathers them into output groups (per shard, or per request when merged != 0)
-cudaError_t launch_plan(const int32_t* seq_lens, int B, int N, int I, int q_len, int merged, int granule,
-                        int min_chunk, int target_units, int n_hb, void* ws, int max_units, int max_split, int hq,
-                        int dv, int64_t* finish_ns, int* status, cudaStream_t s);
+// (merged output only) shards [shard_lo, shard_hi) are decoded
+cudaError_t launch_plan(const int32_t* seq_lens, int B, int N, int I, int q_len, int merged, int shard_lo,
+                        int shard_hi, int granule, int min_chunk, int target_units, int n_hb, void* ws, int max_units,
+                        int max_split, int hq, int dv, int64_t* finish_ns, int* status, cudaStream_t s);
 
 // decode kernels; each returns cudaErrorNotSupported for shapes it does not cover
 enum class DecodePath { GqaSimt, GqaMma, MlaSimt, MlaUmma };
@@ -65,5 +67,7 @@ cudaError_t launch_decode_mla_fp8(const DecodeGeometry& g, const DecodeArgs& a, 
 
 cudaError_t launch_merge(int N, int B, int H, int Dv, const float* o_partial, const float* lse, float* out,
                          float* lse_out, cudaStream_t s);
+cudaError_t launch_lse_rescale(int N, int rank, int B, int H, int Dv, const float* lse_all, const float* o,
+                               float* o_rs, float* lse_out, cudaStream_t s);
 
 }  // namespace dcp

@@ -51,7 +51,48 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
     }
 }
 
+// One rank's share of the merge across GPUs, between the all-gather of the
+// LSEs and the reduce-scatter of the outputs: with every shard's LSE of row
+// (b, h) at hand, LSE = M + ln sum_n exp(lse_n - M), and this rank's partial
+// enters the sum with weight exp(lse_rank - LSE).  The weighted row goes to the
+// reduce-scatter layout [N][B][H/N][Dv] (block n holds the heads rank n keeps).
+__global__ void __launch_bounds__(32 * kMergeWarps)
+    lse_rescale_kernel(int N, int rank, int B, int H, int Dv, const float* __restrict__ lse_all,
+                       const float* __restrict__ o, float* __restrict__ o_rs, float* __restrict__ lse_out) {
+    const int64_t BH = (int64_t)B * H;
+    const int64_t row = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
+    const int lane = threadIdx.x & 31;
+    if (row >= BH) return;
+    float M = -INFINITY;
+    for (int n = 0; n < N; n++) M = fmaxf(M, __ldg(lse_all + (int64_t)n * BH + row));
+    float L = -INFINITY, w = 0.f;
+    if (M != -INFINITY) {
+        float sum = 0.f;
+        for (int n = 0; n < N; n++) sum += expf(__ldg(lse_all + (int64_t)n * BH + row) - M);
+        L = M + logf(sum);
+        const float lr = __ldg(lse_all + (int64_t)rank * BH + row);
+        w = lr == -INFINITY ? 0.f : expf(lr - L);
+    }
+    if (lane == 0 && lse_out) lse_out[row] = L;
+    const int b = (int)(row / H), h = (int)(row - (int64_t)b * H);
+    const int Hn = H / N;
+    const float4* src = reinterpret_cast<const float4*>(o + row * Dv);
+    float4* dst = reinterpret_cast<float4*>(o_rs + (((int64_t)(h / Hn) * B + b) * Hn + h % Hn) * Dv);
+    for (int v = lane; v < Dv / 4; v += 32) {
+        const float4 x = __ldg(src + v);
+        dst[v] = make_float4(w * x.x, w * x.y, w * x.z, w * x.w);
+    }
+}
+
 }  // namespace
+
+cudaError_t launch_lse_rescale(int N, int rank, int B, int H, int Dv, const float* lse_all, const float* o,
+                               float* o_rs, float* lse_out, cudaStream_t s) {
+    const int64_t BH = (int64_t)B * H;
+    const int64_t blocks = (BH + kMergeWarps - 1) / kMergeWarps;
+    lse_rescale_kernel<<<(unsigned)blocks, 32 * kMergeWarps, 0, s>>>(N, rank, B, H, Dv, lse_all, o, o_rs, lse_out);
+    return cudaGetLastError();
+}
 
 cudaError_t launch_merge(int N, int B, int H, int Dv, const float* o_partial, const float* lse, float* out,
                          float* lse_out, cudaStream_t s) {

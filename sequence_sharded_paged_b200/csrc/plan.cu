@@ -12,11 +12,15 @@
 // Context Workloads", section 4.1, which the all-gather + reduce-scatter of
 // the pages performs across GPUs):
 //  - per-shard partials: one group per (n, b), output row block n*B + b;
-//  - merged output: one group per request b over the chunks of ALL its shards,
-//    output row block b.  The group's units are listed next to each other, so
-//    they run at the same time on different SMs and the merging unit finds
-//    their partials still in L2.  Empty shards add no unit; a request with no
-//    token at all gets one empty unit (O = 0, LSE = -inf).
+//  - merged output: one group per request b, output row block b, merged in two
+//    levels: the last chunk of a shard cut into several chunks merges that
+//    shard's chunks, and the last shard of the request to complete merges the
+//    shards' partials.  No merge reads more than max(chunks per shard, N)
+//    partials, so a long request does not leave one CTA a merge of hundreds.
+//    The request's units are listed next to each other, so they run at the
+//    same time on different SMs and the merges find the partials still in L2.
+//    Empty shards add no unit; a request with no token at all gets one empty
+//    unit (O = 0, LSE = -inf).
 #include "common.cuh"
 #include "kernels.h"
 
@@ -57,14 +61,15 @@ __device__ int block_scan_incl(int v, int* total, int* warp_sums) {
 }
 
 __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __restrict__ seq_lens, int B, int N, int I,
-                                                            int q_len, int merged, int granule, int min_chunk,
-                                                            int target_units, int n_hb, uint8_t* ws, WsLayout lay,
-                                                            int64_t* finish_ns, int* status) {
+                                                            int q_len, int merged, int shard_lo, int shard_hi,
+                                                            int granule, int min_chunk, int target_units, int n_hb,
+                                                            uint8_t* ws, WsLayout lay, int64_t* finish_ns,
+                                                            int* status) {
     PlanHeader* hdr = reinterpret_cast<PlanHeader*>(ws);
     Unit* units = reinterpret_cast<Unit*>(ws + lay.off_units);
     int32_t* done = reinterpret_cast<int32_t*>(ws + lay.off_done);
     int32_t* grp_k = reinterpret_cast<int32_t*>(ws + lay.off_k);       // units per group [groups]
-    int32_t* slot_base = reinterpret_cast<int32_t*>(ws + lay.off_base);  // [groups]
+    int32_t* slot_base = reinterpret_cast<int32_t*>(ws + lay.off_base);  // first split slot per group
 
     __shared__ unsigned long long s_total;
     __shared__ int s_hist[33];
@@ -99,10 +104,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
     C = (C + granule - 1) / granule * granule;
     if (C > (1 << 30)) C = 1 << 30;
 
-    // 3. units per group, split-slot scan, length histogram (a group's units share
+    // 3. units per group, split-slot scan, length histogram (a request's units share
     //    one bucket in merged mode: that of its longest unit)
     const int NG = merged ? B : N * B;
-    for (int i = tid; i < NG * n_hb; i += kPlanThreads) done[i] = 0;
+    for (int i = tid; i < (N + 1) * B * n_hb; i += kPlanThreads) done[i] = 0;
     if (finish_ns)
         for (int i = tid; i < NG; i += kPlanThreads) finish_ns[i] = 0;
     int units_local = 0;
@@ -112,13 +117,20 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
         int k = 0, split = 0;
         if (gi < NG) {
             if (merged) {
+                // slots: one per shard with tokens when there are two or more, plus one per
+                // chunk of every shard cut into several chunks
                 const int L = max(seq_lens[gi], 0);
                 int64_t cmax = 0;
-                for (int n = 0; n < N; n++) {
+                int m = 0;
+                for (int n = shard_lo; n < shard_hi; n++) {
                     const int64_t cnt = count_of(L, N, I, n);
-                    k += (int)((cnt + C - 1) / C);
+                    const int kn = (int)((cnt + C - 1) / C);
+                    k += kn;
+                    split += kn >= 2 ? kn : 0;
+                    m += cnt > 0 ? 1 : 0;
                     cmax = cnt > cmax ? cnt : cmax;
                 }
+                split += m >= 2 ? m : 0;
                 if (k == 0) k = 1;
                 atomicAdd(&s_hist[cmax > 0 ? length_bucket(cmax < C ? cmax : C) : 32], k);
             } else {
@@ -134,7 +146,7 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
                 }
             }
             grp_k[gi] = k;
-            split = k >= 2 ? k : 0;
+            if (!merged) split = k >= 2 ? k : 0;
             units_local += k;
         }
         int total;
@@ -172,35 +184,49 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
         for (int b = tid; b < B; b += kPlanThreads) {
             const int L = max(seq_lens[b], 0);
             const int k = grp_k[b];
-            const int sb = slot_base[b];
             int64_t cmax = 0;
-            for (int n = 0; n < N; n++) {
+            int m = 0;
+            for (int n = shard_lo; n < shard_hi; n++) {
                 const int64_t cnt = count_of(L, N, I, n);
                 cmax = cnt > cmax ? cnt : cmax;
+                m += cnt > 0 ? 1 : 0;
             }
-            int pos = atomicAdd(&s_cursor[cmax > 0 ? length_bucket(cmax < C ? cmax : C) : 32], k);
+            const int pos = atomicAdd(&s_cursor[cmax > 0 ? length_bucket(cmax < C ? cmax : C) : 32], k);
             Unit u;
             u.b = b;
-            u.n_chunks = k;
-            u.slot_base = k >= 2 ? sb : -1;
             u.grp = b;
+            u.n_sh = m >= 2 ? m : 1;
+            u.sslot_base = m >= 2 ? slot_base[b] : -1;
+            u.pad = 0;
             if (cmax == 0) {  // a request with no token: one empty unit
-                u.n = 0;
+                u.n = shard_lo;
                 u.t0 = u.t1 = 0;
                 u.slot = -1;
+                u.n_chunks = 1;
+                u.slot_base = -1;
+                u.sslot = -1;
                 units[pos] = u;
                 continue;
             }
-            int j = 0;
-            for (int n = 0; n < N; n++) {
+            int next_slot = slot_base[b] + (m >= 2 ? m : 0);  // chunk slots follow the shard slots
+            int j = 0, i = 0;
+            for (int n = shard_lo; n < shard_hi; n++) {
                 const int64_t cnt = count_of(L, N, I, n);
-                for (int64_t t0 = 0; t0 < cnt; t0 += C, j++) {
-                    u.n = n;
+                if (cnt == 0) continue;
+                const int kn = (int)((cnt + C - 1) / C);
+                u.n = n;
+                u.n_chunks = kn;
+                u.slot_base = kn >= 2 ? next_slot : -1;
+                u.sslot = m >= 2 ? slot_base[b] + i : -1;
+                for (int c = 0; c < kn; c++, j++) {
+                    const int64_t t0 = (int64_t)c * C;
                     u.t0 = (int32_t)t0;
                     u.t1 = (int32_t)(t0 + C < cnt ? t0 + C : cnt);
-                    u.slot = k >= 2 ? sb + j : -1;
+                    u.slot = kn >= 2 ? next_slot + c : -1;
                     units[pos + j] = u;
                 }
+                if (kn >= 2) next_slot += kn;
+                i++;
             }
         }
         return;
@@ -224,6 +250,10 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
             u.n_chunks = k;
             u.slot_base = k >= 2 ? sb : -1;
             u.grp = s;
+            u.sslot = -1;
+            u.n_sh = 1;
+            u.sslot_base = -1;
+            u.pad = 0;
             units[pos] = u;
         }
     }
@@ -231,12 +261,12 @@ __global__ void __launch_bounds__(kPlanThreads) plan_kernel(const int32_t* __res
 
 }  // namespace
 
-cudaError_t launch_plan(const int32_t* seq_lens, int B, int N, int I, int q_len, int merged, int granule,
-                        int min_chunk, int target_units, int n_hb, void* ws, int max_units, int max_split, int hq,
-                        int dv, int64_t* finish_ns, int* status, cudaStream_t s) {
+cudaError_t launch_plan(const int32_t* seq_lens, int B, int N, int I, int q_len, int merged, int shard_lo,
+                        int shard_hi, int granule, int min_chunk, int target_units, int n_hb, void* ws, int max_units,
+                        int max_split, int hq, int dv, int64_t* finish_ns, int* status, cudaStream_t s) {
     WsLayout lay = ws_layout(N, B, hq, dv, max_units, max_split);
-    plan_kernel<<<1, kPlanThreads, 0, s>>>(seq_lens, B, N, I, q_len, merged, granule, min_chunk, target_units, n_hb,
-                                           reinterpret_cast<uint8_t*>(ws), lay, finish_ns, status);
+    plan_kernel<<<1, kPlanThreads, 0, s>>>(seq_lens, B, N, I, q_len, merged, shard_lo, shard_hi, granule, min_chunk,
+                                           target_units, n_hb, reinterpret_cast<uint8_t*>(ws), lay, finish_ns, status);
     return cudaGetLastError();
 }
 

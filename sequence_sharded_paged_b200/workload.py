@@ -16,8 +16,8 @@ import torch
 import synth
 import synth.device as sdev
 
-from . import (DCP_BF16, DCP_FP8_E4M3, DCP_GQA, DCP_MLA, CacheDesc, dcp_decode_workspace_size, dcp_kv_append,
-               dcp_shard_counts, make_cache_desc)
+from . import (DCP_BF16, DCP_FP8_E4M3, DCP_GQA, DCP_MLA, CacheDesc, dcp_decode_workspace_size,
+               dcp_decode_workspace_size_ex, dcp_kv_append, dcp_kv_append_rank, dcp_shard_counts, make_cache_desc)
 
 
 @dataclass
@@ -31,6 +31,7 @@ class DeviceWorkload:
     num_pages: int
     seq_lens: torch.Tensor       # int32 [B] on device
     ws: torch.Tensor             # decode workspace (uint8)
+    rank: int | None = None      # rank-local cache: only shard `rank`'s pages and tables
 
     @property
     def kv_bytes(self) -> int:
@@ -50,13 +51,18 @@ def pages_needed(counts: np.ndarray, page_size: int) -> np.ndarray:
 
 
 def build(w: synth.Workload, counts_with_growth: np.ndarray, fill: bool = True, slack_pages: int = 0,
-          max_rows_per_append: int = 1 << 21) -> DeviceWorkload:
+          max_rows_per_append: int = 1 << 21, rank: int | None = None) -> DeviceWorkload:
     """Allocate the pools and block tables for ``w`` (per-shard counts
     ``counts_with_growth`` [N][B] sized for the longest length the run will
-    reach) and, if ``fill``, append every position [0, L_b) of every request."""
+    reach) and, if ``fill``, append every position [0, L_b) of every request.
+    rank = r: the cache of rank r of an N-GPU group (pages and block tables of
+    shard r only, filled through dcp_kv_append_rank from every position)."""
     dev = torch.device("cuda")
     N, B, P = w.n_shards, w.B, w.page_size
-    need = pages_needed(np.asarray(counts_with_growth), P)
+    counts_with_growth = np.asarray(counts_with_growth)
+    if rank is not None:
+        counts_with_growth = counts_with_growth[rank:rank + 1]
+    need = pages_needed(counts_with_growth, P)
     bt_np, num_pages = synth.deal_block_tables(w.seed_len, need, slack_pages=slack_pages)
     bt = torch.as_tensor(bt_np, device=dev)
     kind = DCP_GQA if w.kind == "gqa" else DCP_MLA
@@ -77,11 +83,11 @@ def build(w: synth.Workload, counts_with_growth: np.ndarray, fill: bool = True, 
                            num_pages=num_pages, hq=w.hq, hkv=w.hkv, dk=w.dk, dv=w.dv, scale=w.scale, batch=B,
                            block_tables=bt, k_pages=k_pages, v_pages=v_pages, kv_scales=kv_scales)
     seq_lens = torch.as_tensor(np.asarray(w.lengths, dtype=np.int32), device=dev)
-    ws_bytes = dcp_decode_workspace_size(desc, B)
+    ws_bytes = dcp_decode_workspace_size(desc, B) if rank is None else dcp_decode_workspace_size_ex(desc, B, 1, 2)
     if ws_bytes == 0:
         raise ValueError("unsupported cache descriptor for decode")
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
-    dw = DeviceWorkload(w, desc, k_pages, v_pages, kv_scales, bt, num_pages, seq_lens, ws)
+    dw = DeviceWorkload(w, desc, k_pages, v_pages, kv_scales, bt, num_pages, seq_lens, ws, rank)
     if fill:
         append_positions(dw, np.zeros(B, np.int64), np.asarray(w.lengths, np.int64), max_rows_per_append)
     return dw
@@ -107,8 +113,10 @@ def append_positions(dw: DeviceWorkload, start: np.ndarray, stop: np.ndarray, ma
         pos = pos_all[lo:hi].contiguous()
         if w.kind == "gqa":
             k, v = sdev.gqa_rows(w.seed_val, req, pos, w.hkv, w.dk)
+        else:
+            k, v = sdev.latent_rows(w.seed_val, req, pos), None
+        if dw.rank is None:
             dcp_kv_append(dw.desc, req, pos, k, v)
         else:
-            lat = sdev.latent_rows(w.seed_val, req, pos)
-            dcp_kv_append(dw.desc, req, pos, lat)
+            dcp_kv_append_rank(dw.desc, dw.rank, req, pos, k, v)
     torch.cuda.synchronize()

@@ -45,8 +45,10 @@ def run_merged(dw, step=0, finish=False):
 
 MERGED_CASES = [
     # (kind, dtype, hq, hkv, D, page, N, I, lengths): every kernel family, empty requests,
-    # shards without tokens, requests split into many chunks
+    # shards without tokens, shards cut into many chunks (both merge levels)
     ("gqa", "bf16", 8, 2, 64, 16, 2, 1, [300, 1000, 0, 1]),              # CUDA-core GQA
+    ("gqa", "bf16", 8, 2, 64, 16, 2, 1, [20_000, 7, 0]),                 # shards of ~20 chunks
+    ("gqa", "bf16", 64, 4, 128, 16, 2, 16, [20_000, 5, 1]),              # tensor-core GQA, ~10 chunks
     ("gqa", "bf16", 64, 4, 128, 16, 8, 128, [1, 200, 3000, 130, 0, 5000]),  # tensor-core GQA
     ("gqa", "bf16", 32, 2, 128, 64, 3, 16, [17, 64, 4100, 2]),
     ("mla", "bf16", 16, 1, 576, 512, 64, 2, 1, [900, 3000, 1, 0]),        # tcgen05 bf16
@@ -54,6 +56,7 @@ MERGED_CASES = [
     ("mla", "fp8", 64, 1, 576, 512, 64, 4, 16, [5000, 333, 2048, 0, 1]),  # tcgen05 fp8
     ("mla", "fp8", 32, 1, 576, 512, 64, 8, 64, [30_000, 100, 9]),
     ("mla", "bf16", 16, 1, 576, 512, 16, 2, 1, [1, 200, 3000]),           # CUDA-core MLA (page 16)
+    ("mla", "bf16", 64, 1, 576, 512, 64, 8, 1, [200_000, 50, 3]),         # 8 shards of ~12 chunks each
 ]
 
 
