@@ -5,7 +5,7 @@ One step = one pass of the whole hot path over the batch, for one new token
 per request:
   dcp_shard_map (owner/slot of position L_b)  ->  dcp_kv_append (write the new
   token into its owner's page)  ->  dcp_decode_merged (every shard's partial
-  attention over positions [0, L_b + 1) and the LSE merge, fused).
+  attention over positions [0, L_b + 1), then the LSE merge, in one call).
 Lengths grow by one token per step, as in decoding.
 
 Metric: KV GB/s = (sum_b attended tokens x KV bytes per token) / step time,
@@ -21,8 +21,6 @@ Qwen3-shaped, MLA Kimi-shaped bf16) are measured the same way under
   - "bands": per-request completion time inside the full batch, by request
     length band (<32k, 32-64k, 64-128k, 128-200k, 200k+), from the device
     timestamps dcp_decode_merged records per request;
-  - "fused_vs_unfused": dcp_decode_merged against dcp_decode_partial +
-    dcp_merge on the same inputs;
   - "e2e": the same step through the C ABI with host buffers, the inputs copied
     in and the output copied out every step on copy streams overlapped with
     the previous / next step's compute.
@@ -217,9 +215,9 @@ def traffic_key(cfg, w) -> str:
 
 
 def launches_per_step(w) -> int:
-    """Kernels one step launches: shard map, append, plan, [query split], decode (merged)."""
+    """Kernels one step launches: shard map, append, plan, [query split], decode, merge."""
     fp8_tc = w.kind == "mla" and w.dtype == "fp8" and w.hq in (16, 32, 64) and w.page_size == 64
-    return 5 if fp8_tc else 4
+    return 6 if fp8_tc else 5
 
 
 def combine_ranks(dist, device, times, sums):
@@ -350,7 +348,7 @@ def measure(args, cfg, rank, world, local_rank, headline):
     bytes_timed = sum(kv_tok[args.warmup + i] for i in range(args.steps)) * bpt
 
     # extra launches on the last timed step's inputs (untimed in `value`): per-request
-    # completion times, and the fused call against partial + merge
+    # completion times
     last = args.warmup + args.steps - 1
     reps = 5
     bands = None
@@ -361,24 +359,6 @@ def measure(args, cfg, rank, world, local_rank, headline):
         torch.cuda.synchronize()
         finish_ms = np.median(fin.cpu().numpy(), axis=0) / 1e6
         bands = band_latency(np.asarray(w.lengths) + last + 1, finish_ms, float(np.median(kern_ms)), bpt)
-    ws_p = torch.empty(dcp.dcp_decode_workspace_size(dw.desc, B), dtype=torch.uint8, device=dev)
-    o_part = torch.empty((N, B, w.hq, w.dv), dtype=torch.float32, device=dev)
-    lse_p = torch.empty((N, B, w.hq), dtype=torch.float32, device=dev)
-    fu = {}
-    for name, fn in (("merged", lambda: dcp.dcp_decode_merged(dw.desc, qs[last], lens_s[last], out, lse_out, ws)),
-                     ("partial_plus_merge", lambda: (dcp.dcp_decode_partial(dw.desc, qs[last], lens_s[last], o_part,
-                                                                            lse_p, ws_p),
-                                                     dcp.dcp_merge(o_part, lse_p, out, lse_out)))):
-        fn()
-        e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        e0.record(stream)
-        for _ in range(reps):
-            fn()
-        e1.record(stream)
-        torch.cuda.synchronize()
-        fu[name + "_ms"] = round(e0.elapsed_time(e1) / reps, 4)
-    del o_part, lse_p, ws_p
-
     # end to end through the C ABI with host buffers: each step's inputs (q, new token
     # rows, positions, lengths) are copied in from pinned memory on one copy stream and
     # its output (out + lse) copied back on another, double-buffered so that the copies
@@ -472,12 +452,11 @@ def measure(args, cfg, rank, world, local_rank, headline):
         "roofline": {"bound": "hbm", "achieved": round(achieved, 1), "peak": hbm, "unit": "GB/s",
                      "frac": round(achieved / hbm, 3), "traffic": traffic,
                      "algorithmic_bytes_per_launch": int(per_launch_bytes),
-                     "kernel": "dcp_decode_merged (planner + split-KV attention + in-kernel LSE merge)",
+                     "kernel": "dcp_decode_merged (planner, [fp8 query split], split-KV attention, LSE merge)",
                      "peak_source": f"{peak_kind} hbm_gbs (MEASURED_PEAKS.json)" if peak_kind == "measured"
                      else "fallback 6650 GB/s (no MEASURED_PEAKS.json)"},
         "clocks": clk,
         "gpu_launches": launches_per_step(w) * args.steps,
-        "fused_vs_unfused": fu,
         "fill_seconds": round(fill_s, 2),
     }
     if bands is not None:

@@ -238,14 +238,15 @@ dcp_status dcp_decode_partial_multi(const dcp_cache_desc* cache, int32_t B, int3
                                     void* stream);
 
 /*
- * dcp_decode_merged -- every shard's partial attention AND the LSE merge in
- * one launch sequence: the output of dcp_decode_partial(_multi) followed by
- * dcp_merge, without the per-shard partials ever being written as a whole.
+ * dcp_decode_merged -- every shard's partial attention and the LSE merge in
+ * one call: the output of dcp_decode_partial(_multi) followed by dcp_merge,
+ * with the per-shard partials kept in the workspace (and dropped from L2 by
+ * the merge once read) instead of the caller's memory.
  * Passage: blog section 4.1 (each GPU's partial output and LSE, reweighted by
  * the LSE values and summed by the all-gather + reduce-scatter).  Here all
- * shards are on one GPU: the chunks of every shard of a request form one merge
- * group, run side by side, and the last of them to finish merges the group's
- * partials while they are still in L2 (then drops them from L2).
+ * shards are on one GPU; the merge runs as a second kernel after the decode
+ * (the kernel boundary orders the partials' stores before the merge reads
+ * them, which costs less than ordering them inside the decode kernel).
  *  q_len, q, seq_lens   as dcp_decode_partial_multi (q_len = 1: one query
  *             token per request, q bf16 [B][hq][dk]).
  *  out        fp32 [B][q_len][hq][dv]: sum over shards of exp(lse_n - LSE) o_n,
@@ -254,11 +255,13 @@ dcp_status dcp_decode_partial_multi(const dcp_cache_desc* cache, int32_t B, int3
  *  lse_out    fp32 [B][q_len][hq]: LSE = M + ln sum_n exp(lse_n - M),
  *             M = max_n lse_n; -inf where a query token attends no position.
  *  finish_ns  int64 [B] or NULL: nanoseconds (device global timer) from the
- *             start of the call's first kernel until request b's output was
- *             stored.  For per-request latency within one batch; the values
- *             order the requests' completions, they are not a kernel timer.
+ *             start of the call's first kernel until the last shard of request
+ *             b was decoded (its merged output follows in the merge kernel).
+ *             For per-request latency within one batch; the values order the
+ *             requests' completions, they are not a kernel timer.
  *  ws, ws_bytes  workspace of at least dcp_decode_workspace_size_ex(cache, B,
- *             q_len, 1) bytes; clobbered.  Concurrent calls need distinct
+ *             q_len, 1) bytes, which includes the partials (4 * N * B * q_len *
+ *             hq * (dv + 1) bytes); clobbered.  Concurrent calls need distinct
  *             workspaces.
  * Errors as dcp_decode_partial (finish_ns must be 16-byte aligned too).
  */

@@ -128,12 +128,18 @@ dcp_status check_desc(const dcp_cache_desc* c, bool need_pools) {
     return DCP_OK;
 }
 
+// What a decode call produces: every shard's partial (the caller's o_partial /
+// lse), the merged output (per-shard partials in the workspace, then the LSE
+// merge), or one rank's shard of a multi-GPU group.
+enum PlanMode { kModePartial = 0, kModeMerged = 1, kModeRank = 2 };
+
 struct Plan {
     DecodeGeometry g;
     WsLayout lay;
     size_t off_qs = 0, off_qinv = 0;  // fp8 MLA query split (0 when unused)
+    size_t off_part = 0, off_part_lse = 0;  // merged mode: the per-shard partials
     int q_len = 1;                    // query tokens per request (rows = q_len * hq)
-    int merged = 0;                   // 1: one output group per request
+    int mode = kModePartial;
 };
 
 constexpr int kMaxQueryLen = 64;
@@ -148,29 +154,30 @@ void add_query_split(const dcp_cache_desc* c, int B, Plan* p) {
     p->lay.total = align256(p->off_qinv + (size_t)B * 64 * sizeof(float));
 }
 
-// Split slots: chunk slots only for shards longer than one chunk, which gives
-// at most 2 * target + 2 of them; merged outputs add one slot per shard with
-// tokens (at most N * B).
-int64_t split_bound(int64_t target, int64_t n_shard_slots, int merged) {
-    return 2 * target + 2 + (merged ? n_shard_slots : 0);
-}
-
 // The plan of a decode of B requests with q_len query tokens each (q_len * hq
-// query rows); merged != 0 gathers every shard of a request into one output
-// group.  Several query tokens are served by the tensor-core paths only.
-bool make_plan(const dcp_cache_desc* c, int B, int q_len, int merged, int num_sms, Plan* p) {
-    if (q_len < 1 || q_len > kMaxQueryLen) return false;
+// query rows) in the given mode.  Several query tokens are served by the
+// tensor-core paths only.  Split slots are needed only for shards longer than
+// one chunk: at most 2 * target + 2 of them.
+bool make_plan(const dcp_cache_desc* c, int B, int q_len, int mode, int num_sms, Plan* p) {
+    if (q_len < 1 || q_len > kMaxQueryLen || mode < kModePartial || mode > kModeRank) return false;
     const int rows = q_len * c->hq;
     if (!decode_geometry(c->kind, c->dtype, rows, c->hkv, c->dk, c->dv, c->page_size, num_sms, &p->g)) return false;
     if (q_len > 1 && p->g.path != DecodePath::GqaMma && p->g.path != DecodePath::MlaUmma) return false;
+    const int shards = mode == kModeRank ? 1 : c->n_shards;
     const int64_t target = (int64_t)p->g.units_per_cta * p->g.ctas;
-    const int64_t max_units = (int64_t)c->n_shards * B + target + 1;
-    const int64_t max_split = split_bound(target, (int64_t)c->n_shards * B, merged);
+    const int64_t max_units = (int64_t)shards * B + target + 1;
+    const int64_t max_split = 2 * target + 2;
     if (max_units > (1 << 30)) return false;
-    p->lay = ws_layout(c->n_shards, B, rows, c->dv, (int)max_units, (int)max_split);
+    p->lay = ws_layout(shards, B, rows, c->dv, (int)max_units, (int)max_split);
     p->q_len = q_len;
-    p->merged = merged;
+    p->mode = mode;
     add_query_split(c, B, p);
+    p->off_part = p->off_part_lse = 0;
+    if (mode == kModeMerged) {
+        p->off_part = p->lay.total;
+        p->off_part_lse = align256(p->off_part + sizeof(float) * (size_t)shards * B * rows * c->dv);
+        p->lay.total = align256(p->off_part_lse + sizeof(float) * (size_t)shards * B * rows);
+    }
     return true;
 }
 
@@ -200,7 +207,7 @@ dcp_status decode_scratch(uint8_t** out) {
 // split slots), repeated down to one unit per CTA.  The bounds are make_plan's
 // for the smaller target.  False when nothing fits.
 bool make_plan_within(const dcp_cache_desc* c, int B, int num_sms, size_t cap, Plan* p) {
-    if (!make_plan(c, B, 1, 0, num_sms, p)) return false;
+    if (!make_plan(c, B, 1, kModePartial, num_sms, p)) return false;
     while (p->lay.total > cap && p->g.units_per_cta > 1) {
         p->g.units_per_cta /= 2;
         const int64_t target = (int64_t)p->g.units_per_cta * p->g.ctas;
@@ -214,15 +221,15 @@ bool make_plan_within(const dcp_cache_desc* c, int B, int num_sms, size_t cap, P
 // The launch sequence of the decode (plan kernel, decode kernel) on a workspace
 // `w` laid out by `p`.
 // rank >= 0: the cache holds only shard `rank`'s block tables, and only that
-// shard is decoded (merged plans only).
+// shard is decoded.
 dcp_status decode_on(const dcp_cache_desc* cache, int32_t B, const void* q, const int32_t* seq_lens,
                      float* o_partial, float* lse, uint8_t* w, const Plan& p, int* status, cudaStream_t s,
                      int64_t* finish_ns = nullptr, int rank = -1) {
     const int64_t target = (int64_t)p.g.units_per_cta * p.g.ctas;
     const int rows = p.q_len * cache->hq;
     const int shard_lo = rank >= 0 ? rank : 0, shard_hi = rank >= 0 ? rank + 1 : cache->n_shards;
-    cudaError_t e = launch_plan(seq_lens, B, cache->n_shards, cache->interleave, p.q_len, p.merged, shard_lo,
-                                shard_hi, p.g.granule, p.g.min_chunk, (int)target, p.g.n_hb, w, p.lay.max_units,
+    cudaError_t e = launch_plan(seq_lens, B, cache->n_shards, cache->interleave, p.q_len, shard_lo, shard_hi,
+                                p.g.granule, p.g.min_chunk, (int)target, p.g.n_hb, w, p.lay.max_units,
                                 p.lay.max_split, rows, cache->dv, finish_ns, status, s);
     if (e != cudaSuccess) return DCP_ERR_CUDA;
     DecodeArgs a;
@@ -430,7 +437,7 @@ size_t dcp_decode_workspace_size(const dcp_cache_desc* cache, int32_t B) {
     int num_sms = 0;
     if (device_info(nullptr, &num_sms) != DCP_OK) return 0;
     Plan p;
-    if (!make_plan(cache, B, 1, 0, num_sms, &p)) return 0;
+    if (!make_plan(cache, B, 1, kModePartial, num_sms, &p)) return 0;
     return p.lay.total;
 }
 
@@ -439,8 +446,7 @@ size_t dcp_decode_workspace_size_ex(const dcp_cache_desc* cache, int32_t B, int3
     int num_sms = 0;
     if (device_info(nullptr, &num_sms) != DCP_OK) return 0;
     Plan p;
-    // mode 2 (one rank's shard) plans like the merged output over fewer shards
-    if (merged < 0 || merged > 2 || !make_plan(cache, B, q_len, merged ? 1 : 0, num_sms, &p)) return 0;
+    if (!make_plan(cache, B, q_len, merged, num_sms, &p)) return 0;
     return p.lay.total;
 }
 
@@ -455,14 +461,14 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
     st = device_info(&status, &num_sms);
     if (st != DCP_OK) return st;
     Plan p;
-    if (!make_plan(cache, B, 1, 0, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
+    if (!make_plan(cache, B, 1, kModePartial, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
     if (ws_bytes < p.lay.total) return DCP_ERR_WORKSPACE_TOO_SMALL;
     return decode_on(cache, B, q, seq_lens, o_partial, lse, static_cast<uint8_t*>(ws), p, status, (cudaStream_t)stream);
 }
 
 // Shared checks and launch of the decode calls that take a query length
 // (rank >= 0: only that shard, from a cache holding only its tables).
-static dcp_status decode_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_len, int merged, const void* q,
+static dcp_status decode_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_len, int mode, const void* q,
                             const int32_t* seq_lens, float* out, float* lse, int64_t* finish_ns, void* ws,
                             size_t ws_bytes, void* stream, int rank = -1) {
     dcp_status st = check_desc(cache, true);
@@ -477,28 +483,39 @@ static dcp_status decode_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_le
     st = device_info(&status, &num_sms);
     if (st != DCP_OK) return st;
     Plan p;
-    if (!make_plan(cache, B, q_len, merged, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
+    if (!make_plan(cache, B, q_len, mode, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
     if (ws_bytes < p.lay.total) return DCP_ERR_WORKSPACE_TOO_SMALL;
-    return decode_on(cache, B, q, seq_lens, out, lse, static_cast<uint8_t*>(ws), p, status, (cudaStream_t)stream,
-                     finish_ns, rank);
+    uint8_t* w = static_cast<uint8_t*>(ws);
+    if (mode != kModeMerged)
+        return decode_on(cache, B, q, seq_lens, out, lse, w, p, status, (cudaStream_t)stream, finish_ns, rank);
+    // merged output: every shard's partial into the workspace, then the LSE merge; the
+    // kernel boundary orders the partials' stores before the merge reads them, and the
+    // merge drops the partials' lines from L2 once read
+    const int rows = q_len * cache->hq;
+    float* part = reinterpret_cast<float*>(w + p.off_part);
+    float* part_lse = reinterpret_cast<float*>(w + p.off_part_lse);
+    st = decode_on(cache, B, q, seq_lens, part, part_lse, w, p, status, (cudaStream_t)stream, finish_ns);
+    if (st != DCP_OK) return st;
+    return cuda_err(launch_merge(cache->n_shards, B, rows, cache->dv, part, part_lse, out, lse, true,
+                                 (cudaStream_t)stream));
 }
 
 dcp_status dcp_decode_partial_multi(const dcp_cache_desc* cache, int32_t B, int32_t q_len, const void* q,
                                     const int32_t* seq_lens, float* o_partial, float* lse, void* ws, size_t ws_bytes,
                                     void* stream) {
-    return decode_ex(cache, B, q_len, 0, q, seq_lens, o_partial, lse, nullptr, ws, ws_bytes, stream);
+    return decode_ex(cache, B, q_len, kModePartial, q, seq_lens, o_partial, lse, nullptr, ws, ws_bytes, stream);
 }
 
 dcp_status dcp_decode_merged(const dcp_cache_desc* cache, int32_t B, int32_t q_len, const void* q,
                              const int32_t* seq_lens, float* out, float* lse_out, int64_t* finish_ns, void* ws,
                              size_t ws_bytes, void* stream) {
-    return decode_ex(cache, B, q_len, 1, q, seq_lens, out, lse_out, finish_ns, ws, ws_bytes, stream);
+    return decode_ex(cache, B, q_len, kModeMerged, q, seq_lens, out, lse_out, finish_ns, ws, ws_bytes, stream);
 }
 
 dcp_status dcp_decode_rank(const dcp_cache_desc* cache, int32_t rank, int32_t B, int32_t q_len, const void* q,
                            const int32_t* seq_lens, float* o, float* lse, void* ws, size_t ws_bytes, void* stream) {
     if (!cache || rank < 0) return DCP_ERR_INVALID_ARG;
-    return decode_ex(cache, B, q_len, 1, q, seq_lens, o, lse, nullptr, ws, ws_bytes, stream, rank);
+    return decode_ex(cache, B, q_len, kModeRank, q, seq_lens, o, lse, nullptr, ws, ws_bytes, stream, rank);
 }
 
 // No workspace argument and no allocation: for callers that cannot allocate
@@ -517,7 +534,7 @@ dcp_status dcp_decode_partial_noalloc(const dcp_cache_desc* cache, int32_t B, co
     st = device_info(&status, &num_sms);
     if (st != DCP_OK) return st;
     Plan p;
-    if (!make_plan(cache, B, 1, 0, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
+    if (!make_plan(cache, B, 1, kModePartial, num_sms, &p)) return DCP_ERR_UNSUPPORTED;
     if (!make_plan_within(cache, B, num_sms, DCP_STATIC_SCRATCH_BYTES, &p)) return DCP_ERR_WORKSPACE_TOO_SMALL;
     uint8_t* w = nullptr;
     st = decode_scratch(&w);
@@ -529,7 +546,7 @@ dcp_status dcp_merge(int32_t N, int32_t B, int32_t H, int32_t Dv, const float* o
                      float* out, float* lse_out, void* stream) {
     if (N < 1 || B < 1 || H < 1 || Dv < 4 || Dv % 4 || !o_partial || !lse || !out) return DCP_ERR_INVALID_ARG;
     if (!aligned16(o_partial) || !aligned16(out)) return DCP_ERR_MISALIGNED;
-    return cuda_err(launch_merge(N, B, H, Dv, o_partial, lse, out, lse_out, (cudaStream_t)stream));
+    return cuda_err(launch_merge(N, B, H, Dv, o_partial, lse, out, lse_out, false, (cudaStream_t)stream));
 }
 
 dcp_status dcp_lse_rescale(int32_t N, int32_t rank, int32_t B, int32_t H, int32_t Dv, const float* lse_all,

@@ -159,20 +159,15 @@ __device__ __forceinline__ float fast_exp2(float x) {
 // work units produced by the planner
 // ---------------------------------------------------------------------------
 struct Unit {
-    int32_t n;           // shard
-    int32_t b;           // request
-    int32_t t0, t1;      // local token range [t0, t1) of shard n of request b
-    int32_t slot;        // chunk slot of this unit, -1 when its shard is one unit
-    int32_t n_chunks;    // units (chunks) of this unit's shard
-    int32_t slot_base;   // first chunk slot of the shard
-    int32_t grp;         // output row block: n*B + b (per-shard partials) or b (merged output)
-    int32_t sslot;       // merged output: slot of this shard's partial in its request's merge,
-                         // -1 when the request has a single shard with tokens (or per-shard outputs)
-    int32_t n_sh;        // merged output: shards with tokens in the request (else 1)
-    int32_t sslot_base;  // merged output: first shard slot of the request
-    int32_t pad;
+    int32_t n;          // shard
+    int32_t b;          // request
+    int32_t t0, t1;     // local token range [t0, t1) of shard n of request b
+    int32_t slot;       // split-partial slot of this chunk, -1 when the shard is one chunk
+    int32_t n_chunks;   // chunks of this shard
+    int32_t slot_base;  // first split slot of this shard
+    int32_t grp;        // output row block of this shard: (n - first decoded shard) * B + b
 };
-static_assert(sizeof(Unit) == 48, "Unit layout");
+static_assert(sizeof(Unit) == 32, "Unit layout");
 
 struct PlanHeader {
     int32_t num_units;
@@ -181,7 +176,7 @@ struct PlanHeader {
     int32_t max_split;
     int64_t total_tokens;
     int32_t next_unit;  // dynamic-scheduling ticket (zeroed by the planner)
-    int32_t merged;     // 1: one output group per request (all shards merged)
+    int32_t pad;
     int64_t t_start_ns; // %globaltimer when the planner started
 };
 
@@ -203,10 +198,9 @@ constexpr int kStageLast = 2;
 constexpr int kStageValid = 4;
 
 // Workspace layout (all offsets 256-byte aligned):
-//   PlanHeader | Unit[max_units] | int32 done[(N+1)*B*hq] | int32 shard_k[N*B] |
+//   PlanHeader | Unit[max_units] | int32 done[N*B*hq] | int32 shard_k[N*B] |
 //   int32 slot_base[N*B] | float split_o[max_split][hq][dv] | float split_lse[max_split][hq]
-// done: counters per (shard, request, head block) for the chunks of a shard,
-// then per (request, head block) for the shards of a request (merged output).
+// done: chunk counters per (shard, request, head block).
 struct WsLayout {
     size_t off_units, off_done, off_k, off_base, off_split_o, off_split_lse, total;
     int32_t max_units, max_split;
@@ -219,8 +213,8 @@ __host__ inline WsLayout ws_layout(int N, int B, int hq, int dv, int max_units, 
     size_t o = align256(sizeof(PlanHeader));
     w.off_units = o;
     o = align256(o + sizeof(Unit) * (size_t)max_units);
-    w.off_done = o;  // counters per (shard or request, head block); head blocks <= hq
-    o = align256(o + sizeof(int32_t) * (size_t)(N + 1) * B * hq);
+    w.off_done = o;  // one counter per (shard, request, head block); head blocks <= hq
+    o = align256(o + sizeof(int32_t) * (size_t)N * B * hq);
     w.off_k = o;
     o = align256(o + sizeof(int32_t) * (size_t)N * B);
     w.off_base = o;
@@ -263,7 +257,7 @@ struct DecodeArgs {
     // several query tokens per request: hq counts query ROWS (q_len x heads), row
     // r = j * (hq / q_len) + head belongs to query token j
     int32_t q_len;
-    int64_t* finish_ns;  // per output group: ns from the planner's start to its final output (or null)
+    int64_t* finish_ns;  // per request: ns from the planner's start until its last shard is decoded (or null)
     // first shard whose block tables are present: 0 when block_tables holds every
     // shard ([N][B][max_local_pages]); r when it holds only shard r's ([1][B][..]),
     // the cache of rank r of a multi-GPU group
@@ -279,12 +273,12 @@ __device__ __forceinline__ int row_limit(const DecodeArgs& a, const Unit& u, int
     return L <= 0 ? 0 : (int)count_of(L, a.n_shards, a.interleave, u.n);
 }
 
-// Completion time of output group `grp` (call after a part of its final output
-// is stored; the planner zeroes the array and the last part to finish sets it).
-__device__ __forceinline__ void record_finish(const DecodeArgs& a, int grp) {
+// Completion time of request b (call after a shard's result of b is stored; the
+// planner zeroes the array and the last shard to finish sets it).
+__device__ __forceinline__ void record_finish(const DecodeArgs& a, int b) {
     if (!a.finish_ns) return;
     const uint64_t dt = global_timer_ns() - (uint64_t)a.plan->t_start_ns;
-    atomicMax(reinterpret_cast<unsigned long long*>(a.finish_ns + grp), (unsigned long long)dt);
+    atomicMax(reinterpret_cast<unsigned long long*>(a.finish_ns + b), (unsigned long long)dt);
 }
 
 // Invalidate the 128-byte L2 line at p (128-byte aligned) without writing it

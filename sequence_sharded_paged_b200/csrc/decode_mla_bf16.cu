@@ -25,16 +25,13 @@
 // maximum is rescaled lazily: O^T is rescaled only when a head's maximum grows
 // by more than 2^8 (P then stays below 256).
 //
-// Warp roles (256 threads, one CTA per SM, persistent, units taken from an
+// Warp roles (224 threads, one CTA per SM, persistent, units taken from an
 // atomic ticket):
 //   warp 0      TMA producer (lane 0): nine [64][64] boxes per tile, 128 B swizzle
 //   warp 1      TMEM allocation; lane 0 issues the S MMAs of each tile
 //   warps 2..5  softmax, lazy rescale of O^T, epilogue (one per TMEM lane
 //               quadrant; lanes l and l + 16 share head l's 64 tokens)
 //   warp 6      lane 0 issues the P V MMAs of each tile
-//   warp 7      merges: when a unit completes a shard cut into several chunks, or the
-//               last shard of a request (merged output), the softmax warps queue the
-//               merge here and go on with the next unit
 #include "common.cuh"
 #include "finish.cuh"
 #include "kernels.h"
@@ -70,9 +67,7 @@ constexpr int kQBytes = kKB * 64 * 128;   // Q padded to 64 rows: 73728
 constexpr int kStages = 2;
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kSmBar = 1;                 // named barrier of the softmax warps
-constexpr int kThreads = 256;              // producer, S issuer, softmax x 4, P V issuer, merge
-constexpr int kMergeWarp = 7;
-constexpr int kMQ = 8;                     // merge-warp jobs in flight
+constexpr int kThreads = 224;              // producer, S issuer, softmax x 4, P V issuer
 constexpr int kPBytes = 64 * 128;         // P_lo^T [64 heads][64 tokens] bf16
 
 constexpr uint32_t kOffQ = 0;
@@ -80,8 +75,7 @@ constexpr uint32_t kOffTiles = kQBytes;
 constexpr uint32_t kOffPlo = kOffTiles + kStages * kTileBytes;
 constexpr uint32_t kOffBars = kOffPlo + kPBytes;
 constexpr uint32_t kOffMeta = kOffBars + 32 * 8;
-constexpr uint32_t kOffQueue = kOffMeta + kStages * 16;  // int2 [kMQ]: (job, unit)
-constexpr uint32_t kOffSmall = kOffQueue + kMQ * 8;
+constexpr uint32_t kOffSmall = kOffMeta + kStages * 16;
 constexpr uint32_t kSmemBytes = kOffSmall + (3 * 64 + 16) * 4 + 1024;
 
 enum : int {
@@ -94,14 +88,7 @@ enum : int {
     B_Q_FREE = 13,
     B_O_FREE = 14,
     B_FINAL = 15,
-    B_MQ_FULL = 16,   // [kMQ]
-    B_MQ_EMPTY = 24,  // [kMQ]
 };
-static_assert(B_MQ_EMPTY + kMQ <= 32 && B_MQ_FULL + kMQ <= B_MQ_EMPTY, "barrier area");
-
-// merge-warp jobs: count a stored unit result in (and merge what it completes);
-// -1 ends the warp
-enum : int { kJobEnd = -1, kJobCount = 1 };
 
 __device__ __forceinline__ uint32_t sw128(int row, int chunk) {
     return (uint32_t)(row * 128 + (((chunk ^ row) & 7) << 4));
@@ -136,7 +123,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* s_misc = reinterpret_cast<int*>(s_alpha + 64);  // [0] tmem base, [2] split flag, [3] abort
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_misc + 3);
 
-    int2* mqueue = reinterpret_cast<int2*>(sm + kOffQueue);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t sm_u32 = smem_u32(sm);
 
@@ -152,10 +138,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar + B_Q_FREE, 1);
         mbar_init(bar + B_O_FREE, 4);
         mbar_init(bar + B_FINAL, 2);
-        for (int i = 0; i < kMQ; i++) {
-            mbar_init(bar + B_MQ_FULL + i, 1);
-            mbar_init(bar + B_MQ_EMPTY + i, 1);
-        }
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -315,51 +297,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma::commit(bar + B_FINAL);
             mbar_wait(bar + B_FINAL, 0, nullptr, a.status);
         }
-    } else if (warp == kMergeWarp) {
-        // ------------------------------------------------------------------ merges
-        for (uint32_t mk = 0;; mk++) {
-            const int qi = (int)(mk % kMQ);
-            int ok = 1;
-            if (lane == 0) ok = mbar_wait(bar + B_MQ_FULL + qi, (mk / kMQ) & 1, s_abort, a.status);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            const volatile int* jq = reinterpret_cast<const volatile int*>(mqueue + qi);
-            const int2 job = make_int2(jq[0], jq[1]);
-            if (job.x == kJobEnd) break;
-            const Unit u = a.units[job.y];
-            // The softmax warps stored the unit's result and synchronised before queueing
-            // it; this fence (release is cumulative) makes those stores visible to the
-            // other CTAs before the counter says they are there.
-            __threadfence();
-            bool complete = true;
-            if (u.slot >= 0) {  // a chunk of a shard cut into several: the last one merges them
-                int last = 0;
-                if (lane == 0) last = atomicAdd(shard_counter(a, u, 0, 1), 1) == u.n_chunks - 1;
-                complete = __shfl_sync(0xffffffffu, last, 0);
-                if (complete) {
-                    __threadfence();
-                    float *so, *sl;
-                    shard_dst(a, u, &so, &sl);
-                    merge_slots(a, u.slot_base, u.n_chunks, 0, HQ, so, sl, 0, 1, lane);
-                    __threadfence();
-                    __syncwarp();
-                }
-            }
-            if (complete && u.sslot >= 0) {  // a shard of a request of several: the last one merges them
-                int last = 0;
-                if (lane == 0) last = atomicAdd(request_counter(a, u, 0, 1), 1) == u.n_sh - 1;
-                complete = __shfl_sync(0xffffffffu, last, 0);
-                if (complete) {
-                    __threadfence();
-                    merge_slots(a, u.sslot_base, u.n_sh, 0, HQ, a.o_partial + (int64_t)u.grp * a.hq * 512,
-                                a.lse + (int64_t)u.grp * a.hq, 0, 1, lane);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) {
-                if (complete) record_finish(a, u.grp);
-                mbar_arrive(bar + B_MQ_EMPTY + qi);
-            }
-        }
     } else {
         // ------------------------------------------------------------------ softmax / epilogue
         // A failed (timed-out) wait sets `fail`; the four warps learn it at the
@@ -376,8 +313,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t seq = 0, unit_k = 0;
         float m_used = -INFINITY, lsum = 0.f;
         int lim = 0x7fffffff;  // local tokens [0, lim) of the unit's shard this row attends
-        int ui = 0;            // index of the current unit
-        uint32_t mjobs = 0;    // merge jobs queued (thread tid 0)
         bool o_has = false;
         bool fail = false;
         Unit u{};
@@ -394,8 +329,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const bool last = meta.flags & kStageLast;
             const int nvalid = (meta.flags >> 8) & 0xFF;
             if (first) {
-                ui = meta.unit;
-                u = a.units[ui];
+                u = a.units[meta.unit];
                 lim = head ? row_limit(a, u, h / (HQ / a.q_len)) : 0x7fffffff;
                 // Q of request u.b: all S MMAs of the previous unit are complete (first unit passes)
                 fail = !mbar_wait(bar + B_Q_FREE, (unit_k & 1) ^ 1, s_abort, a.status);
@@ -526,8 +460,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 const float l = lsum + __shfl_xor_sync(0xffffffffu, lsum, 16);  // both halves of the head
                 if (head && half == 0) s_l[h] = l > 0.f ? 1.f / l : 0.f;      // O = O^T * (1 / l)
                 if (named_barrier_or(kSmBar, 128, fail)) break;
-                float *obase, *lbase;
-                unit_dst(a, u, &obase, &lbase);
+                const int64_t grp = u.grp;
+                const bool split = u.n_chunks > 1;
+                float* obase = split ? a.split_o + (int64_t)u.slot * a.hq * 512 : a.o_partial + grp * a.hq * 512;
+                float* lbase = split ? a.split_lse + (int64_t)u.slot * a.hq : a.lse + grp * a.hq;
 #pragma unroll 1
                 for (int blk = 0; blk < 4; blk++) {
                     const int dv = blk * 128 + 32 * qd + lane;
@@ -545,32 +481,28 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar + B_O_FREE);
-                if (u.slot >= 0 || u.sslot >= 0) {
-                    // the merge warp counts this result in (and merges what it completes), so
-                    // these warps go on without waiting for the stores to drain
+                if (split) {
+                    // the last unit of the group to finish merges the group's split partials
+                    __threadfence();
                     named_barrier_sync(kSmBar, 128);
-                    if (tid == 0) {
-                        const int qi = (int)(mjobs % kMQ);
-                        if (mbar_wait(bar + B_MQ_EMPTY + qi, ((mjobs / kMQ) & 1) ^ 1, s_abort, a.status)) {
-                            mqueue[qi] = make_int2(kJobCount, ui);
-                            mbar_arrive(bar + B_MQ_FULL + qi);
-                            mjobs++;
+                    if (tid == 0) s_misc[2] = (atomicAdd(a.done + grp, 1) == u.n_chunks - 1) ? 1 : 0;
+                    named_barrier_sync(kSmBar, 128);
+                    const int is_last = *reinterpret_cast<volatile int*>(s_misc + 2);
+                    named_barrier_sync(kSmBar, 128);
+                    if (is_last) {
+                        __threadfence();
+                        merge_slots(a, u.slot_base, u.n_chunks, 0, HQ, shard_out(a, u), shard_lse(a, u), tid >> 5, 4, tid & 31);
+                        if (a.finish_ns) {
+                            named_barrier_sync(kSmBar, 128);
+                            if (tid == 0) record_finish(a, u.b);
                         }
                     }
                 } else if (a.finish_ns) {
                     named_barrier_sync(kSmBar, 128);
-                    if (tid == 0) record_finish(a, u.grp);
+                    if (tid == 0) record_finish(a, u.b);
                 }
             }
             seq++;
-        }
-        // no more units: end the merge warp once it has taken every queued job
-        if (tid == 0 && !*s_abort) {
-            const int qi = (int)(mjobs % kMQ);
-            if (mbar_wait(bar + B_MQ_EMPTY + qi, ((mjobs / kMQ) & 1) ^ 1, s_abort, a.status)) {
-                mqueue[qi] = make_int2(kJobEnd, 0);
-                mbar_arrive(bar + B_MQ_FULL + qi);
-            }
         }
     }
 

@@ -48,10 +48,6 @@
 //               32..63; g also picks the value blocks 2 g, 2 g + 1 that the warp
 //               rescales and stores.
 //   warp 10     issues P V of each tile
-//   warp 11     merges: when a unit completes a shard cut into several chunks, or the
-//               last shard of a request (merged output), the softmax warps queue the
-//               merge here and go on with the next unit; this warp reads the partials
-//               (still in L2 as a rule), writes the merged result and discards them.
 #include "common.cuh"
 #include "finish.cuh"
 #include "kernels.h"
@@ -92,9 +88,7 @@ constexpr int kPBuf = 2 * kPPage;          // a tile of two pages: 16 KB
 constexpr float kRescaleLog2 = 8.f;
 constexpr int kSmBar = 1;                  // the 256 softmax threads
 constexpr int kSoftWarps = 8;
-constexpr int kThreads = 32 * (4 + kSoftWarps);  // producer, S issuer, softmax x 8, P V issuer, merge
-constexpr int kMergeWarp = 3 + kSoftWarps;
-constexpr int kMQ = 8;                     // merge-warp jobs in flight
+constexpr int kThreads = 32 * (3 + kSoftWarps);  // producer, S issuer, softmax x 8, P V issuer
 constexpr uint32_t kColO = 0, kColS = 256, kColQ = 384;  // TMEM columns
 
 constexpr uint32_t kOffTiles = 0;
@@ -102,9 +96,8 @@ constexpr uint32_t kOffRope = kOffTiles + kSlots * kTileBytes;
 constexpr uint32_t kOffP = kOffRope + kRopeBytes;
 constexpr uint32_t kOffScales = kOffP + 2 * kPBuf;
 constexpr uint32_t kOffBars = kOffScales + kSlots * kPg * 4;
-constexpr uint32_t kOffMeta = kOffBars + 48 * 8;
-constexpr uint32_t kOffQueue = kOffMeta + kSlots * 16;  // int2 [kMQ]: (job, unit)
-constexpr uint32_t kOffSmall = kOffQueue + kMQ * 8;
+constexpr uint32_t kOffMeta = kOffBars + 32 * 8;
+constexpr uint32_t kOffSmall = kOffMeta + kSlots * 16;
 // s_alpha[64], s_inv[64], s_gmax[2][64], s_gl[2][64], misc[16]
 constexpr uint32_t kSmemBytes = kOffSmall + (6 * 64 + 16) * 4 + 1024;
 static_assert(kSmemBytes <= 232448, "shared memory budget");
@@ -121,14 +114,7 @@ enum : int {
     B_Q_FREE = 25,
     B_O_FREE = 26,
     B_FINAL = 27,
-    B_MQ_FULL = 32,   // [kMQ]
-    B_MQ_EMPTY = 40,  // [kMQ]
 };
-static_assert(B_MQ_EMPTY + kMQ <= 48 && B_MQ_FULL + kMQ <= B_MQ_EMPTY, "barrier area");
-
-// merge-warp jobs: count a stored unit result in (and merge what it completes);
-// -1 ends the warp
-enum : int { kJobEnd = -1, kJobCount = 1 };
 
 // Page (= tile) k of the ring sequence uses slot k mod 5 and completes phase (k / 5) & 1
 // of that slot's barriers.
@@ -262,7 +248,6 @@ __global__ void __launch_bounds__(kThreads, 1)
     int* s_misc = reinterpret_cast<int*>(s_gl + 128);  // [0] tmem base, [2] split flag, [3] abort
     volatile int* s_abort = reinterpret_cast<volatile int*>(s_misc + 3);
 
-    int2* mqueue = reinterpret_cast<int2*>(sm + kOffQueue);
     const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
     const uint32_t sm_u32 = smem_u32(sm);
 
@@ -281,10 +266,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         mbar_init(bar + B_Q_FREE, 1);
         mbar_init(bar + B_O_FREE, kSoftWarps);
         mbar_init(bar + B_FINAL, 2);
-        for (int i = 0; i < kMQ; i++) {
-            mbar_init(bar + B_MQ_FULL + i, 1);
-            mbar_init(bar + B_MQ_EMPTY + i, 1);
-        }
         *s_abort = 0;
         fence_barrier_init();
     }
@@ -472,51 +453,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             umma::commit(bar + B_FINAL);
             mbar_wait(bar + B_FINAL, 0, nullptr, a.status);
         }
-    } else if (warp == kMergeWarp) {
-        // ------------------------------------------------------------------ merges
-        for (uint32_t mk = 0;; mk++) {
-            const int qi = (int)(mk % kMQ);
-            int ok = 1;
-            if (lane == 0) ok = mbar_wait(bar + B_MQ_FULL + qi, (mk / kMQ) & 1, s_abort, a.status);
-            if (!__shfl_sync(0xffffffffu, ok, 0)) break;
-            const volatile int* jq = reinterpret_cast<const volatile int*>(mqueue + qi);
-            const int2 job = make_int2(jq[0], jq[1]);
-            if (job.x == kJobEnd) break;
-            const Unit u = a.units[job.y];
-            // The softmax warps stored the unit's result and synchronised before queueing
-            // it; this fence (release is cumulative) makes those stores visible to the
-            // other CTAs before the counter says they are there.
-            __threadfence();
-            bool complete = true;
-            if (u.slot >= 0) {  // a chunk of a shard cut into several: the last one merges them
-                int last = 0;
-                if (lane == 0) last = atomicAdd(shard_counter(a, u, 0, 1), 1) == u.n_chunks - 1;
-                complete = __shfl_sync(0xffffffffu, last, 0);
-                if (complete) {
-                    __threadfence();
-                    float *so, *sl;
-                    shard_dst(a, u, &so, &sl);
-                    merge_slots(a, u.slot_base, u.n_chunks, 0, HQ, so, sl, 0, 1, lane);
-                    __threadfence();
-                    __syncwarp();
-                }
-            }
-            if (complete && u.sslot >= 0) {  // a shard of a request of several: the last one merges them
-                int last = 0;
-                if (lane == 0) last = atomicAdd(request_counter(a, u, 0, 1), 1) == u.n_sh - 1;
-                complete = __shfl_sync(0xffffffffu, last, 0);
-                if (complete) {
-                    __threadfence();
-                    merge_slots(a, u.sslot_base, u.n_sh, 0, HQ, a.o_partial + (int64_t)u.grp * a.hq * 512,
-                                a.lse + (int64_t)u.grp * a.hq, 0, 1, lane);
-                }
-            }
-            __syncwarp();
-            if (lane == 0) {
-                if (complete) record_finish(a, u.grp);
-                mbar_arrive(bar + B_MQ_EMPTY + qi);
-            }
-        }
     } else {
         // ------------------------------------------------------------------ query rows, softmax, epilogue
         const int qd = warp & 3;                  // TMEM lane quadrant
@@ -532,8 +468,6 @@ __global__ void __launch_bounds__(kThreads, 1)
         uint32_t seq = 0, kk = 0, unit_k = 0;
         float m_used = -INFINITY, lpart = 0.f, f = 0.f;
         int lim = 0x7fffffff;  // local tokens [0, lim) of the unit's shard this row attends
-        int ui = 0;            // index of the current unit
-        uint32_t mjobs = 0;    // merge jobs queued (thread tid 0)
         bool o_has = false, fail = false;
         Unit u{};
         while (true) {
@@ -557,8 +491,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             const int nvalid = mine ? (((wg ? m1.flags : m0.flags) >> 8) & 0xFF) : 0;
             const bool page_full = nvalid == kPg;
             if (first) {
-                ui = m0.unit;
-                u = a.units[ui];
+                u = a.units[m0.unit];
                 f = head ? __ldg(a.qinv + (int64_t)u.b * 64 + h) * a.scale_log2 : 0.f;
                 lim = head ? row_limit(a, u, h / (HQ / a.q_len)) : 0x7fffffff;
                 // the previous unit's S MMAs are complete (first unit passes at once)
@@ -772,8 +705,10 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma::fence_after_sync();
                 const float lg = lpart + __shfl_xor_sync(0xffffffffu, lpart, 16);  // this token group
                 if (half == 0) s_gl[wg * 64 + h] = lg;
-                float *obase, *lbase;
-                unit_dst(a, u, &obase, &lbase);
+                const int64_t grp = u.grp;
+                const bool split = u.n_chunks > 1;
+                float* obase = split ? a.split_o + (int64_t)u.slot * a.hq * 512 : a.o_partial + grp * a.hq * 512;
+                float* lbase = split ? a.split_lse + (int64_t)u.slot * a.hq : a.lse + grp * a.hq;
                 if (named_barrier_or(kSmBar, 256, fail)) break;
                 if (head && half == 0 && wg == 0) {
                     const float l = lg + s_gl[64 + h];
@@ -800,35 +735,30 @@ __global__ void __launch_bounds__(kThreads, 1)
                 umma::fence_before_sync();
                 __syncwarp();
                 if (lane == 0) mbar_arrive(bar + B_O_FREE);
-                if (u.slot >= 0 || u.sslot >= 0) {
-                    // the merge warp counts this result in (and merges what it completes), so
-                    // these warps go on without waiting for the stores to drain
+                if (split) {
+                    __threadfence();
                     named_barrier_sync(kSmBar, 256);
-                    if (tid == 0) {
-                        const int qi = (int)(mjobs % kMQ);
-                        if (mbar_wait(bar + B_MQ_EMPTY + qi, ((mjobs / kMQ) & 1) ^ 1, s_abort, a.status)) {
-                            mqueue[qi] = make_int2(kJobCount, ui);
-                            mbar_arrive(bar + B_MQ_FULL + qi);
-                            mjobs++;
+                    if (tid == 0) s_misc[2] = (atomicAdd(a.done + grp, 1) == u.n_chunks - 1) ? 1 : 0;
+                    named_barrier_sync(kSmBar, 256);
+                    const int is_last = *reinterpret_cast<volatile int*>(s_misc + 2);
+                    named_barrier_sync(kSmBar, 256);
+                    if (is_last) {
+                        __threadfence();
+                        merge_slots(a, u.slot_base, u.n_chunks, 0, HQ, shard_out(a, u), shard_lse(a, u), tid >> 5, 8, tid & 31);
+                        if (a.finish_ns) {
+                            named_barrier_sync(kSmBar, 256);
+                            if (tid == 0) record_finish(a, u.b);
                         }
                     }
                 } else if (a.finish_ns) {
                     named_barrier_sync(kSmBar, 256);
-                    if (tid == 0) record_finish(a, u.grp);
+                    if (tid == 0) record_finish(a, u.b);
                 }
                 if (threadIdx.x == 64) TRACE(13, seq);
             }
             if (threadIdx.x == 64) TRACE(11, seq);
             seq++;
             kk += pair ? 2 : 1;
-        }
-        // no more units: end the merge warp once it has taken every queued job
-        if (tid == 0 && !*s_abort) {
-            const int qi = (int)(mjobs % kMQ);
-            if (mbar_wait(bar + B_MQ_EMPTY + qi, ((mjobs / kMQ) & 1) ^ 1, s_abort, a.status)) {
-                mqueue[qi] = make_int2(kJobEnd, 0);
-                mbar_arrive(bar + B_MQ_FULL + qi);
-            }
         }
     }
 

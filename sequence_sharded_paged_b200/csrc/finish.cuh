@@ -1,10 +1,8 @@
-// finish.cuh -- end of one work unit: store the unit's output when its group
-// has one unit, or its split partial and, in the last unit of the group to
-// finish, the LSE merge of the group's units.  A group is the chunks of one
-// shard (per-shard partials, the split-KV reduce) or the chunks of every
-// shard of one request (merged output).  The merge is the arithmetic of
+// finish.cuh -- end of one work unit: store a shard's partial, or a chunk's
+// split partial and, in the last chunk of the shard to finish, the LSE merge
+// of the chunks (split-KV reduce).  The merge is the arithmetic of
 // "Efficient Decode Context Parallelism with vLLM for Long Context Workloads",
-// section 4.1 (LSE-reweighted sum of partials).
+// section 4.1 (LSE-reweighted sum of partials), applied within one shard.
 #pragma once
 
 #include "common.cuh"
@@ -83,94 +81,58 @@ __device__ inline void merge_slots(const DecodeArgs& a, int base, int K, int h0,
     }
 }
 
-// Where a unit's own result goes: its chunk slot when its shard is cut into
-// several chunks; otherwise where its shard's result goes (shard_dst).
-// Where a shard's result goes: its slot in the request's merge (merged output
-// over several shards), else the output row block u.grp.
-__device__ __forceinline__ void shard_dst(const DecodeArgs& a, const Unit& u, float** o, float** lse) {
-    if (u.sslot >= 0) {
-        *o = a.split_o + (int64_t)u.sslot * a.hq * a.dv;
-        *lse = a.split_lse + (int64_t)u.sslot * a.hq;
-    } else {
-        *o = a.o_partial + (int64_t)u.grp * a.hq * a.dv;
-        *lse = a.lse + (int64_t)u.grp * a.hq;
-    }
+// The output row block of the unit's shard.
+__device__ __forceinline__ float* shard_out(const DecodeArgs& a, const Unit& u) {
+    return a.o_partial + (int64_t)u.grp * a.hq * a.dv;
 }
-__device__ __forceinline__ void unit_dst(const DecodeArgs& a, const Unit& u, float** o, float** lse) {
-    if (u.slot >= 0) {
-        *o = a.split_o + (int64_t)u.slot * a.hq * a.dv;
-        *lse = a.split_lse + (int64_t)u.slot * a.hq;
-    } else {
-        shard_dst(a, u, o, lse);
-    }
-}
-// completion counters: the chunks of shard (u.n, u.b), and the shards of request u.b
-__device__ __forceinline__ int32_t* shard_counter(const DecodeArgs& a, const Unit& u, int hb, int n_hb) {
-    return a.done + ((int64_t)u.n * a.batch + u.b) * n_hb + hb;
-}
-__device__ __forceinline__ int32_t* request_counter(const DecodeArgs& a, const Unit& u, int hb, int n_hb) {
-    return a.done + ((int64_t)a.n_shards * a.batch + u.b) * n_hb + hb;
+__device__ __forceinline__ float* shard_lse(const DecodeArgs& a, const Unit& u) {
+    return a.lse + (int64_t)u.grp * a.hq;
 }
 
 // Executed by the NT threads of barrier `bar_id` (tid in [0, NT), NT a
 // multiple of 32).
 //  sO   [nh][dv] normalised output of this unit for rows h0..h0+nh-1 (smem)
 //  sLse [nh]     natural-log LSE (-inf when the unit saw no token)
-//  hb / n_hb     head block of this unit and head blocks per unit (counters are
-//                per (shard or request, head block))
-// Stores the unit's result, then merges its shard's chunks when it completes the
-// shard, then the request's shards when that completes the request (merged
-// output), and records the request's completion time when a.finish_ns is set.
+//  hb / n_hb     head block of this unit and head blocks per unit (split counters
+//                are per (shard, head block))
+// Records the request's completion time (a.finish_ns) when this completes the shard.
 template <int NT>
 __device__ void finish_unit(const DecodeArgs& a, const Unit& u, int hb, int n_hb, int h0, int nh,
                             const float* sO, const float* sLse, int* s_flag, int tid, int bar_id) {
     const int dv = a.dv;
     const int nvec = nh * dv / 4;
-    float* o_dst;
-    float* l_dst;
-    unit_dst(a, u, &o_dst, &l_dst);
-    const bool counted = u.slot >= 0 || u.sslot >= 0;  // does anything merge this result later?
+    if (u.n_chunks == 1) {
+        float4* dst = reinterpret_cast<float4*>(shard_out(a, u) + (int64_t)h0 * dv);
+        const float4* src = reinterpret_cast<const float4*>(sO);
+        for (int i = tid; i < nvec; i += NT) dst[i] = src[i];
+        for (int i = tid; i < nh; i += NT) shard_lse(a, u)[h0 + i] = sLse[i];
+        if (a.finish_ns) {
+            named_barrier_sync(bar_id, NT);
+            if (tid == 0) record_finish(a, u.b);
+        }
+        return;
+    }
     {
-        float4* dst = reinterpret_cast<float4*>(o_dst + (int64_t)h0 * dv);
+        float4* dst = reinterpret_cast<float4*>(a.split_o + ((int64_t)u.slot * a.hq + h0) * dv);
         const float4* src = reinterpret_cast<const float4*>(sO);
         for (int i = tid; i < nvec; i += NT) __stcg(dst + i, src[i]);
-        for (int i = tid; i < nh; i += NT) __stcg(l_dst + h0 + i, sLse[i]);
+        for (int i = tid; i < nh; i += NT) __stcg(a.split_lse + (int64_t)u.slot * a.hq + h0 + i, sLse[i]);
     }
-    bool complete = true;  // has this unit completed its shard (and, without a second level, the request)?
-    if (counted) {
-        __threadfence();
-        named_barrier_sync(bar_id, NT);
-        // level 1: the chunks of the shard
-        if (u.slot >= 0) {
-            if (tid == 0) *s_flag = (atomicAdd(shard_counter(a, u, hb, n_hb), 1) == u.n_chunks - 1) ? 1 : 0;
-            named_barrier_sync(bar_id, NT);
-            complete = *(volatile int*)s_flag;
-            named_barrier_sync(bar_id, NT);
-            if (complete) {
-                __threadfence();
-                float *so, *sl;
-                shard_dst(a, u, &so, &sl);
-                merge_slots(a, u.slot_base, u.n_chunks, h0, nh, so, sl, tid >> 5, NT >> 5, tid & 31);
-                __threadfence();
-                named_barrier_sync(bar_id, NT);
-            }
-        }
-        // level 2: the shards of the request
-        if (complete && u.sslot >= 0) {
-            if (tid == 0) *s_flag = (atomicAdd(request_counter(a, u, hb, n_hb), 1) == u.n_sh - 1) ? 1 : 0;
-            named_barrier_sync(bar_id, NT);
-            complete = *(volatile int*)s_flag;
-            named_barrier_sync(bar_id, NT);
-            if (complete) {
-                __threadfence();
-                merge_slots(a, u.sslot_base, u.n_sh, h0, nh, a.o_partial + (int64_t)u.grp * a.hq * dv,
-                            a.lse + (int64_t)u.grp * a.hq, tid >> 5, NT >> 5, tid & 31);
-            }
-        }
+    __threadfence();
+    named_barrier_sync(bar_id, NT);
+    if (tid == 0) {
+        int old = atomicAdd(a.done + (int64_t)u.grp * n_hb + hb, 1);
+        *s_flag = (old == u.n_chunks - 1) ? 1 : 0;
     }
-    if (complete && a.finish_ns) {
+    named_barrier_sync(bar_id, NT);
+    const int last = *(volatile int*)s_flag;
+    named_barrier_sync(bar_id, NT);
+    if (!last) return;
+    __threadfence();
+    merge_slots(a, u.slot_base, u.n_chunks, h0, nh, shard_out(a, u), shard_lse(a, u), tid >> 5, NT >> 5, tid & 31);
+    if (a.finish_ns) {
         named_barrier_sync(bar_id, NT);
-        if (tid == 0) record_finish(a, u.grp);
+        if (tid == 0) record_finish(a, u.b);
     }
 }
 

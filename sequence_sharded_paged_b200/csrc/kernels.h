@@ -34,11 +34,11 @@ cudaError_t launch_shard_map(int64_t n_pos, const int32_t* pos, const int32_t* r
                              int32_t* local_out, int64_t* slot_out, int* status, cudaStream_t s);
 cudaError_t launch_append(const AppendArgs& a, cudaStream_t s);
 
-// planner: splits every (shard, request) into chunks of at most chunk_tokens and
-// gathers them into output groups (per shard, or per request when merged != 0)
-// (merged output only) shards [shard_lo, shard_hi) are decoded
-cudaError_t launch_plan(const int32_t* seq_lens, int B, int N, int I, int q_len, int merged, int shard_lo,
-                        int shard_hi, int granule, int min_chunk, int target_units, int n_hb, void* ws, int max_units,
+// planner: splits every (shard, request) of shards [shard_lo, shard_hi) into
+// chunks of at most chunk_tokens; output row block of shard n of request b:
+// (n - shard_lo) * B + b
+cudaError_t launch_plan(const int32_t* seq_lens, int B, int N, int I, int q_len, int shard_lo, int shard_hi,
+                        int granule, int min_chunk, int target_units, int n_hb, void* ws, int max_units,
                         int max_split, int hq, int dv, int64_t* finish_ns, int* status, cudaStream_t s);
 
 // decode kernels; each returns cudaErrorNotSupported for shapes it does not cover
@@ -65,8 +65,9 @@ bool mla_umma_supported(int hq, int page_size);
 cudaError_t launch_decode_mla_bf16(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s);
 cudaError_t launch_decode_mla_fp8(const DecodeGeometry& g, const DecodeArgs& a, cudaStream_t s);
 
+// discard != 0: o_partial is scratch whose lines are dropped from L2 once read
 cudaError_t launch_merge(int N, int B, int H, int Dv, const float* o_partial, const float* lse, float* out,
-                         float* lse_out, cudaStream_t s);
+                         float* lse_out, bool discard, cudaStream_t s);
 cudaError_t launch_lse_rescale(int N, int rank, int B, int H, int Dv, const float* lse_all, const float* o,
                                float* o_rs, float* lse_out, cudaStream_t s);
 

@@ -18,7 +18,7 @@ constexpr int kMergeWarps = 8;
 
 __global__ void __launch_bounds__(32 * kMergeWarps)
     merge_kernel(int N, int64_t BH, int Dv, const float* __restrict__ o_part, const float* __restrict__ lse_part,
-                 float* __restrict__ out, float* __restrict__ lse_out) {
+                 float* __restrict__ out, float* __restrict__ lse_out, int discard) {
     const int64_t row = (int64_t)blockIdx.x * kMergeWarps + (threadIdx.x >> 5);
     const int lane = threadIdx.x & 31;
     if (row >= BH) return;
@@ -48,6 +48,13 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
             acc.w = fmaf(w, x.w, acc.w);
         }
         o[v] = acc;
+    }
+    if (discard) {  // the partials are scratch: drop their lines from L2 without writing them back
+        __syncwarp();
+        for (int i = lane; i < N * (Dv / 32); i += 32) {
+            const int n = i / (Dv / 32), l = i - n * (Dv / 32);
+            discard_l2_line(o_part + ((int64_t)n * BH + row) * Dv + l * 32);
+        }
     }
 }
 
@@ -95,10 +102,11 @@ cudaError_t launch_lse_rescale(int N, int rank, int B, int H, int Dv, const floa
 }
 
 cudaError_t launch_merge(int N, int B, int H, int Dv, const float* o_partial, const float* lse, float* out,
-                         float* lse_out, cudaStream_t s) {
+                         float* lse_out, bool discard, cudaStream_t s) {
     const int64_t BH = (int64_t)B * H;
     const int64_t blocks = (BH + kMergeWarps - 1) / kMergeWarps;
-    merge_kernel<<<(unsigned)blocks, 32 * kMergeWarps, 0, s>>>(N, BH, Dv, o_partial, lse, out, lse_out);
+    merge_kernel<<<(unsigned)blocks, 32 * kMergeWarps, 0, s>>>(N, BH, Dv, o_partial, lse, out, lse_out,
+                                                                discard && Dv % 32 == 0 ? 1 : 0);
     return cudaGetLastError();
 }
 

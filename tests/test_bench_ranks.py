@@ -73,10 +73,10 @@ def test_summarize_clocks_keeps_only_the_timed_window():
 
 def test_launch_count_per_path():
     import synth
-    # shard map, append, plan, decode (with the merge inside); fp8 MLA adds the query split
-    assert bench.launches_per_step(synth.workload(5)) == 5
-    assert bench.launches_per_step(synth.workload(4)) == 4
-    assert bench.launches_per_step(synth.workload(3)) == 4
+    # shard map, append, plan, decode, merge; fp8 MLA adds the query split
+    assert bench.launches_per_step(synth.workload(5)) == 6
+    assert bench.launches_per_step(synth.workload(4)) == 5
+    assert bench.launches_per_step(synth.workload(3)) == 5
 
 
 def test_band_latency_summary():
