@@ -30,7 +30,11 @@ Qwen3-shaped, MLA Kimi-shaped bf16) are measured the same way under
 
 Multi-GPU (torchrun, one rank per GPU): each rank runs its own independent
 batch (replicas of the workload, weak scaling); there is no data-path
-collective.  Timing is the max over ranks of the device time.
+collective.  Timing is the max over ranks of the device time.  With
+--dcp-across-gpus the ranks instead form one DCP group: each holds the shard
+of the positions it owns (N = number of GPUs), decodes it, and the partials
+are combined by an all-gather of the LSEs and a reduce-scatter over query
+heads (NCCL); the group decodes one batch (strong scaling).
 """
 from __future__ import annotations
 
@@ -74,6 +78,9 @@ def parse():
     ap.add_argument("--no-bands", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-seconds", type=float, default=25.0, help="target CPU work of the oracle sample")
+    ap.add_argument("--dcp-across-gpus", action="store_true",
+                    help="one shard per rank (N = number of GPUs): rank-local caches and the all-gather / "
+                         "reduce-scatter exchange over NCCL, one batch for the whole group (strong scaling)")
     return ap.parse_args()
 
 
@@ -282,7 +289,7 @@ def measure(args, cfg, rank, world, local_rank, headline):
     fill_s = time.time() - t0
     B, N = w.B, w.n_shards
     L0 = torch.as_tensor(np.asarray(w.lengths, np.int32), device=dev)
-    ws = torch.empty(dcp.dcp_decode_workspace_size_ex(dw.desc, B, 1, True), dtype=torch.uint8, device=dev)
+    ws = torch.empty(dcp.dcp_decode_workspace_size_ex(dw.desc, B, 1, dcp.DCP_DECODE_MERGED), dtype=torch.uint8, device=dev)
 
     # per-step inputs, resident in HBM before the timed region
     qs = [sdev.q(w.seed_val, B, w.hq, w.dk, step=s + 1) for s in range(n_total)]
@@ -471,6 +478,95 @@ def measure(args, cfg, rank, world, local_rank, headline):
     return res, w
 
 
+def measure_dcp(args, cfg, rank, world, local_rank):
+    """One DCP group across the ranks (one shard per GPU): each step appends the new
+    tokens (every rank is given every token and keeps its own) and runs
+    parallel.decode_distributed.  Returns the result dict and the workload."""
+    import torch
+    import torch.distributed as dist
+
+    import sequence_sharded_paged_b200 as dcp
+    import synth.device as sdev
+    from sequence_sharded_paged_b200 import parallel
+    from sequence_sharded_paged_b200 import workload as wl
+
+    dcp.lib()
+    dev = torch.device("cuda", local_rank)
+    w = synth.workload(cfg, n_shards=world, interleave=args.interleave)
+    if args.batch_limit:
+        w.B = min(w.B, args.batch_limit)
+        w.lengths = w.lengths[:w.B]
+    n_total = args.warmup + args.steps
+    counts = wl.gpu_shard_counts(np.asarray(w.lengths) + n_total + 1, world, w.interleave)
+    t0 = time.time()
+    dw = wl.build(w, counts, rank=rank)
+    fill_s = time.time() - t0
+    B = w.B
+    ws = parallel.rank_workspace(dw.desc, B, device=dev)
+    L0 = torch.as_tensor(np.asarray(w.lengths, np.int32), device=dev)
+    qs = [sdev.q(w.seed_val, B, w.hq, w.dk, step=s + 1) for s in range(n_total)]
+    req = torch.arange(B, dtype=torch.int32, device=dev)
+    pos_s = [(L0 + s).contiguous() for s in range(n_total)]
+    lens_s = [(L0 + s + 1).contiguous() for s in range(n_total)]
+    if w.kind == "gqa":
+        new_rows = [sdev.gqa_rows(w.seed_val, req, pos_s[s], w.hkv, w.dk) for s in range(n_total)]
+    else:
+        new_rows = [(sdev.latent_rows(w.seed_val, req, pos_s[s]), None) for s in range(n_total)]
+    stream = torch.cuda.current_stream()
+
+    def step(s):
+        k, v = new_rows[s]
+        dcp.dcp_kv_append_rank(dw.desc, rank, None, pos_s[s], k, v)
+        return parallel.decode_distributed(dw.desc, rank, world, qs[s], lens_s[s], ws)
+
+    clocks = Clocks(local_rank)
+    clocks.start()
+    for s in range(args.warmup):
+        step(s)
+    torch.cuda.synchronize()
+    if dcp.dcp_get_device_status() != dcp.DCP_OK:
+        raise RuntimeError("device status after warm-up")
+    dist.barrier()
+    torch.cuda.synchronize()
+    wall0 = time.time()
+    e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    e0.record(stream)
+    for i in range(args.steps):
+        step(args.warmup + i)
+    e1.record(stream)
+    torch.cuda.synchronize()
+    wall1 = time.time()
+    dist.barrier()
+    clocks.mark(wall0, wall1)
+    clk = clocks.stop()
+    if dcp.dcp_get_device_status() != dcp.DCP_OK:
+        raise RuntimeError("device status after the timed steps")
+    (ms,), _ = combine_ranks(dist, dev, [e0.elapsed_time(e1)], [0])
+    kv_tok = sum(int(np.sum(w.lengths)) + B * (args.warmup + i + 1) for i in range(args.steps))
+    bytes_all = kv_tok * w.kv_bytes_per_token  # the group decodes the batch once per step
+    hbm, peak_kind = peaks()
+    gbs = bytes_all / (ms * 1e-3) / 1e9
+    per_gpu = gbs / world
+    res = {
+        "value": round(gbs, 1), "unit": "GB/s", "ms_per_step": round(ms / args.steps, 4),
+        "steps_per_s": round(args.steps / (ms * 1e-3), 2),
+        "pct_hbm_measured": round(100 * per_gpu / hbm, 1), "pct_hbm_nominal_8tbs": round(100 * per_gpu / 8000.0, 1),
+        "dtype": "bf16" if w.dtype == "bf16" else "fp8_e4m3 cache, bf16 q, fp32 accumulate",
+        "config": workload_config(w, cfg) | {"parallelism": f"DCP across {world} GPU(s): one shard per GPU, "
+                                                             f"all-gather of LSEs + reduce-scatter over heads"},
+        "roofline": {"bound": "hbm", "achieved": round(per_gpu, 1), "peak": hbm, "unit": "GB/s",
+                     "frac": round(per_gpu / hbm, 3), "traffic": None,
+                     "kernel": "whole DCP step per GPU (append, rank decode, exchange)",
+                     "peak_source": f"{peak_kind} hbm_gbs"},
+        "clocks": clk,
+        "gpu_launches": (5 if (w.kind == "mla" and w.dtype == "fp8") else 4) * args.steps,
+        "fill_seconds": round(fill_s, 2),
+    }
+    del dw, ws, qs, new_rows
+    torch.cuda.empty_cache()
+    return res, w
+
+
 # ----------------------------------------------------------------------------
 # the oracle on host cores (CPU baseline / reference arm)
 # ----------------------------------------------------------------------------
@@ -559,18 +655,34 @@ def main():
     import torch
     import torch.distributed as dist
     torch.cuda.set_device(local_rank)
-    if world > 1:
+    if args.dcp_across_gpus and world == 1:
+        # a group of one still runs the exchange through NCCL
+        import socket
+        with socket.socket() as sk:
+            sk.bind(("127.0.0.1", 0))
+            port = sk.getsockname()[1]
+        os.environ.setdefault("MASTER_ADDR", "127.0.0.1")
+        os.environ.setdefault("MASTER_PORT", str(port))
+        os.environ.setdefault("RANK", "0")
+        os.environ.setdefault("WORLD_SIZE", "1")
+    if world > 1 or args.dcp_across_gpus:
         import datetime
-        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=600),
+        # a short timeout ends a rank's collective with an error if another rank has failed
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120 if args.dcp_across_gpus else 600),
                                 device_id=torch.device("cuda", local_rank))
     try:
-        r, w = measure(args, args.config, rank, world, local_rank, True)
+        if args.dcp_across_gpus:
+            r, w = measure_dcp(args, args.config, rank, world, local_rank)
+        else:
+            r, w = measure(args, args.config, rank, world, local_rank, True)
         res = {"metric": METRIC, "value": r["value"], "unit": "GB/s", "n_gpus": world, "steps": args.steps,
                "warmup": args.warmup, "ms_per_step": r["ms_per_step"], "steps_per_s": r["steps_per_s"],
-               "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": r["dtype"],
+               "higher_is_better": True, "scaling": "strong" if args.dcp_across_gpus else "weak",
+               "vs_baseline": None, "dtype": r["dtype"],
                "data": "synthetic (seeded counter-based generator; lengths shaped like the agentic trace)"}
         res.update({k: v for k, v in r.items() if k not in res})
-        others = [int(c) for c in args.per_config.split(",") if c.strip()] if world == 1 else []
+        others = ([int(c) for c in args.per_config.split(",") if c.strip()]
+                  if world == 1 and not args.dcp_across_gpus else [])
         per = {}
         for cfg in others:
             if cfg == args.config:
@@ -585,7 +697,7 @@ def main():
         if rank == 0:
             print(json.dumps(res), flush=True)
     finally:
-        if world > 1:
+        if world > 1 or args.dcp_across_gpus:
             dist.barrier()
             dist.destroy_process_group()
 

@@ -59,6 +59,12 @@ typedef enum {
 } dcp_status;
 
 typedef enum { DCP_GQA = 0, DCP_MLA = 1 } dcp_kind;
+/* what a decode call produces (workspace sizing of dcp_decode_workspace_size_ex) */
+typedef enum {
+    DCP_DECODE_PARTIAL = 0,  /* every shard's partial: dcp_decode_partial(_multi) */
+    DCP_DECODE_MERGED = 1,   /* the merged output: dcp_decode_merged */
+    DCP_DECODE_RANK = 2      /* one rank's shard of a multi-GPU group: dcp_decode_rank */
+} dcp_decode_mode;
 typedef enum { DCP_BF16 = 0, DCP_FP8_E4M3 = 1 } dcp_dtype;
 
 /*
@@ -201,14 +207,13 @@ dcp_status dcp_decode_partial(const dcp_cache_desc* cache, int32_t B, const void
                               float* o_partial, float* lse, void* ws, size_t ws_bytes, void* stream);
 
 /*
- * dcp_decode_workspace_size_ex -- bytes of device workspace that
- * dcp_decode_partial_multi (merged = 0), dcp_decode_merged (merged = 1) or
- * dcp_decode_rank (merged = 2) needs for this cache, batch and query length on
- * the CURRENT device (host function; no GPU work).  Returns 0 for an invalid
- * descriptor, another value of merged, or a shape no kernel of this build
- * covers.
+ * dcp_decode_workspace_size_ex -- bytes of device workspace that the decode
+ * call of `mode` (dcp_decode_mode: dcp_decode_partial(_multi),
+ * dcp_decode_merged or dcp_decode_rank) needs for this cache, batch and query
+ * length on the CURRENT device (host function; no GPU work).  Returns 0 for an
+ * invalid descriptor or mode, or a shape no kernel of this build covers.
  */
-size_t dcp_decode_workspace_size_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_len, int32_t merged);
+size_t dcp_decode_workspace_size_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_len, int32_t mode);
 
 /*
  * dcp_decode_partial_multi -- dcp_decode_partial with q_len query tokens per
@@ -230,7 +235,7 @@ size_t dcp_decode_workspace_size_ex(const dcp_cache_desc* cache, int32_t B, int3
  *             0 where there are none.
  *  lse        fp32 [N][B][q_len][hq]: natural-log LSE, -inf where none.
  *  ws, ws_bytes  workspace of at least dcp_decode_workspace_size_ex(cache, B,
- *             q_len, 0) bytes; clobbered.
+ *             q_len, DCP_DECODE_PARTIAL) bytes; clobbered.
  * Errors as dcp_decode_partial.
  */
 dcp_status dcp_decode_partial_multi(const dcp_cache_desc* cache, int32_t B, int32_t q_len, const void* q,
@@ -260,7 +265,7 @@ dcp_status dcp_decode_partial_multi(const dcp_cache_desc* cache, int32_t B, int3
  *             For per-request latency within one batch; the values order the
  *             requests' completions, they are not a kernel timer.
  *  ws, ws_bytes  workspace of at least dcp_decode_workspace_size_ex(cache, B,
- *             q_len, 1) bytes, which includes the partials (4 * N * B * q_len *
+ *             q_len, DCP_DECODE_MERGED) bytes, which includes the partials (4 * N * B * q_len *
  *             hq * (dv + 1) bytes); clobbered.  Concurrent calls need distinct
  *             workspaces.
  * Errors as dcp_decode_partial (finish_ns must be 16-byte aligned too).
@@ -294,7 +299,7 @@ dcp_status dcp_kv_append_rank(const dcp_cache_desc* cache, int32_t rank, int64_t
  *  o          fp32 [B][q_len][hq][dv]: the normalised partial output, 0 where
  *             the rank owns no attended position.
  *  lse        fp32 [B][q_len][hq]: its natural-log LSE, -inf where none.
- *  ws, ws_bytes  at least dcp_decode_workspace_size_ex(cache, B, q_len, 2).
+ *  ws, ws_bytes  at least dcp_decode_workspace_size_ex(cache, B, q_len, DCP_DECODE_RANK).
  * Next: all-gather lse across the group, dcp_lse_rescale, reduce-scatter.
  * Errors as dcp_decode_partial.
  */

@@ -37,6 +37,10 @@ DCP_MLA = 1
 DCP_BF16 = 0
 DCP_FP8_E4M3 = 1
 
+DCP_DECODE_PARTIAL = 0
+DCP_DECODE_MERGED = 1
+DCP_DECODE_RANK = 2
+
 EXPORTED = ("dcp_status_string", "dcp_shard_counts", "dcp_shard_map", "dcp_kv_append",
             "dcp_decode_workspace_size", "dcp_decode_workspace_size_ex", "dcp_decode_partial",
             "dcp_decode_partial_multi", "dcp_decode_merged", "dcp_decode_partial_noalloc", "dcp_merge",
@@ -158,8 +162,9 @@ def dcp_decode_partial(desc: CacheDesc, q, seq_lens, o_partial, lse, ws, stream=
            "dcp_decode_partial")
 
 
-def dcp_decode_workspace_size_ex(desc: CacheDesc, batch: int, q_len: int = 1, merged: bool = False) -> int:
-    return int(lib().dcp_decode_workspace_size_ex(ctypes.byref(desc), batch, q_len, 1 if merged else 0))
+def dcp_decode_workspace_size_ex(desc: CacheDesc, batch: int, q_len: int = 1, mode: int = DCP_DECODE_PARTIAL) -> int:
+    """Workspace bytes of the decode call of `mode` (DCP_DECODE_PARTIAL, _MERGED or _RANK)."""
+    return int(lib().dcp_decode_workspace_size_ex(ctypes.byref(desc), batch, q_len, int(mode)))
 
 
 def dcp_decode_partial_multi(desc: CacheDesc, q, seq_lens, o_partial, lse, ws, stream=None) -> None:

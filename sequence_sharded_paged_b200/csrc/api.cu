@@ -128,10 +128,10 @@ dcp_status check_desc(const dcp_cache_desc* c, bool need_pools) {
     return DCP_OK;
 }
 
-// What a decode call produces: every shard's partial (the caller's o_partial /
-// lse), the merged output (per-shard partials in the workspace, then the LSE
-// merge), or one rank's shard of a multi-GPU group.
-enum PlanMode { kModePartial = 0, kModeMerged = 1, kModeRank = 2 };
+// What a decode call produces (dcp_decode_mode): every shard's partial (the
+// caller's o_partial / lse), the merged output (per-shard partials in the
+// workspace, then the LSE merge), or one rank's shard of a multi-GPU group.
+enum PlanMode { kModePartial = DCP_DECODE_PARTIAL, kModeMerged = DCP_DECODE_MERGED, kModeRank = DCP_DECODE_RANK };
 
 struct Plan {
     DecodeGeometry g;
@@ -441,12 +441,12 @@ size_t dcp_decode_workspace_size(const dcp_cache_desc* cache, int32_t B) {
     return p.lay.total;
 }
 
-size_t dcp_decode_workspace_size_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_len, int32_t merged) {
+size_t dcp_decode_workspace_size_ex(const dcp_cache_desc* cache, int32_t B, int32_t q_len, int32_t mode) {
     if (check_desc(cache, false) != DCP_OK || B != cache->batch) return 0;
     int num_sms = 0;
     if (device_info(nullptr, &num_sms) != DCP_OK) return 0;
     Plan p;
-    if (!make_plan(cache, B, q_len, merged, num_sms, &p)) return 0;
+    if (!make_plan(cache, B, q_len, mode, num_sms, &p)) return 0;
     return p.lay.total;
 }
 

@@ -17,12 +17,12 @@ from __future__ import annotations
 import torch
 import torch.distributed as dist
 
-from . import CacheDesc, dcp_decode_rank, dcp_decode_workspace_size_ex, dcp_lse_rescale
+from . import DCP_DECODE_RANK, CacheDesc, dcp_decode_rank, dcp_decode_workspace_size_ex, dcp_lse_rescale
 
 
 def rank_workspace(desc: CacheDesc, batch: int, q_len: int = 1, device=None) -> torch.Tensor:
     """Workspace of dcp_decode_rank for this rank's cache."""
-    n = dcp_decode_workspace_size_ex(desc, batch, q_len, 2)
+    n = dcp_decode_workspace_size_ex(desc, batch, q_len, DCP_DECODE_RANK)
     if n == 0:
         raise ValueError("unsupported cache descriptor for dcp_decode_rank")
     return torch.empty(n, dtype=torch.uint8, device=device)

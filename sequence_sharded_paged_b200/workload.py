@@ -16,7 +16,7 @@ import torch
 import synth
 import synth.device as sdev
 
-from . import (DCP_BF16, DCP_FP8_E4M3, DCP_GQA, DCP_MLA, CacheDesc, dcp_decode_workspace_size,
+from . import (DCP_BF16, DCP_DECODE_RANK, DCP_FP8_E4M3, DCP_GQA, DCP_MLA, CacheDesc, dcp_decode_workspace_size,
                dcp_decode_workspace_size_ex, dcp_kv_append, dcp_kv_append_rank, dcp_shard_counts, make_cache_desc)
 
 
@@ -83,7 +83,7 @@ def build(w: synth.Workload, counts_with_growth: np.ndarray, fill: bool = True, 
                            num_pages=num_pages, hq=w.hq, hkv=w.hkv, dk=w.dk, dv=w.dv, scale=w.scale, batch=B,
                            block_tables=bt, k_pages=k_pages, v_pages=v_pages, kv_scales=kv_scales)
     seq_lens = torch.as_tensor(np.asarray(w.lengths, dtype=np.int32), device=dev)
-    ws_bytes = dcp_decode_workspace_size(desc, B) if rank is None else dcp_decode_workspace_size_ex(desc, B, 1, 2)
+    ws_bytes = dcp_decode_workspace_size(desc, B) if rank is None else dcp_decode_workspace_size_ex(desc, B, 1, DCP_DECODE_RANK)
     if ws_bytes == 0:
         raise ValueError("unsupported cache descriptor for decode")
     ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)

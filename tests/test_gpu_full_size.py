@@ -55,7 +55,7 @@ def _build(w):
 def _merged(dw):
     w = dw.w
     q = sdev.q(w.seed_val, w.B, w.hq, w.dk, 0)
-    ws = torch.empty(dcp.dcp_decode_workspace_size_ex(dw.desc, w.B, 1, True), dtype=torch.uint8, device="cuda")
+    ws = torch.empty(dcp.dcp_decode_workspace_size_ex(dw.desc, w.B, 1, dcp.DCP_DECODE_MERGED), dtype=torch.uint8, device="cuda")
     out = torch.full((w.B, w.hq, w.dv), float("nan"), dtype=torch.float32, device="cuda")
     lse = torch.full((w.B, w.hq), float("nan"), dtype=torch.float32, device="cuda")
     dcp.dcp_decode_merged(dw.desc, q, dw.seq_lens, out, lse, ws)

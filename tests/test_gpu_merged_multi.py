@@ -26,7 +26,8 @@ def _clear_status():
 
 
 def _ws(dw, q_len, merged):
-    n = dcp.dcp_decode_workspace_size_ex(dw.desc, dw.w.B, q_len, merged)
+    mode = dcp.DCP_DECODE_MERGED if merged else dcp.DCP_DECODE_PARTIAL
+    n = dcp.dcp_decode_workspace_size_ex(dw.desc, dw.w.B, q_len, mode)
     assert n > 0
     return torch.empty(n, dtype=torch.uint8, device="cuda")
 
@@ -160,8 +161,8 @@ def test_multi_query_unsupported_shapes():
     """Several query tokens are served by the tensor-core kernels only."""
     w = small_workload("gqa", "bf16", [40, 50], 8, 2, 64, 64, 16, 2, 1, seed=55)  # 4 heads per KV head
     dw = build_for_test(w)
-    assert dcp.dcp_decode_workspace_size_ex(dw.desc, w.B, 2, False) == 0  # 8 MMA rows: CUDA-core path
-    assert dcp.dcp_decode_workspace_size_ex(dw.desc, w.B, 4, False) > 0   # 16 rows: tensor cores
+    assert dcp.dcp_decode_workspace_size_ex(dw.desc, w.B, 2, dcp.DCP_DECODE_PARTIAL) == 0  # 8 MMA rows: CUDA-core path
+    assert dcp.dcp_decode_workspace_size_ex(dw.desc, w.B, 4, dcp.DCP_DECODE_PARTIAL) > 0   # 16 rows: tensor cores
     qd, _ = _q_multi(w, 2)
     o = torch.empty((2, w.B, 2, w.hq, w.dv), dtype=torch.float32, device="cuda")
     l = torch.empty((2, w.B, 2, w.hq), dtype=torch.float32, device="cuda")

@@ -157,3 +157,37 @@ def test_decode_host_validation_without_gpu():
 def test_libsynth_exports():
     lib = synth.device_lib()
     assert hasattr(lib, "synth_fill_flat") and hasattr(lib, "synth_fill_kv_rows")
+
+
+def test_new_entry_points_host_validation_without_gpu():
+    """The multi-query, merged and rank calls reject bad arguments with the status include/dcp.h
+    names, before any CUDA call."""
+    L = dcp.lib()
+    A = 1024
+    d = _valid_mla_desc(dcp.DCP_BF16)
+
+    def multi(q_len, B=1, q=A, o=A, lse=A, ws=A):
+        return L.dcp_decode_partial_multi(ctypes.byref(d), B, q_len, q, A, o, lse, ws, 1 << 20, None)
+
+    def merged(q_len, fin=None, B=1):
+        return L.dcp_decode_merged(ctypes.byref(d), B, q_len, A, A, A, A, fin, A, 1 << 20, None)
+
+    def rank(r, q_len=1):
+        return L.dcp_decode_rank(ctypes.byref(d), r, 1, q_len, A, A, A, A, A, 1 << 20, None)
+
+    for f in (multi, merged):
+        assert f(0) == dcp.DCP_ERR_INVALID_ARG        # q_len >= 1
+        assert f(65) == dcp.DCP_ERR_UNSUPPORTED       # q_len <= 64
+        assert f(1, B=2) == dcp.DCP_ERR_INVALID_ARG   # B != cache->batch
+    assert multi(2, q=None) == dcp.DCP_ERR_INVALID_ARG
+    assert multi(2, o=A + 4) == dcp.DCP_ERR_MISALIGNED
+    assert merged(1, fin=A + 8) == dcp.DCP_ERR_MISALIGNED
+    assert rank(-1) == dcp.DCP_ERR_INVALID_ARG
+    assert rank(2) == dcp.DCP_ERR_INVALID_ARG           # rank < n_shards (2)
+    assert L.dcp_kv_append_rank(ctypes.byref(d), 5, 1, None, A, A, None, None) == dcp.DCP_ERR_INVALID_ARG
+    # dcp_lse_rescale: N, rank, B, H, Dv, lse_all, o, o_rs, lse_out
+    assert L.dcp_lse_rescale(2, 0, 1, 3, 64, A, A, A, None, None) == dcp.DCP_ERR_INVALID_ARG   # H % N
+    assert L.dcp_lse_rescale(2, 2, 1, 4, 64, A, A, A, None, None) == dcp.DCP_ERR_INVALID_ARG   # rank < N
+    assert L.dcp_lse_rescale(2, 0, 1, 4, 6, A, A, A, None, None) == dcp.DCP_ERR_INVALID_ARG    # Dv % 4
+    assert L.dcp_lse_rescale(2, 0, 1, 4, 64, A, A + 4, A, None, None) == dcp.DCP_ERR_MISALIGNED
+    assert L.dcp_decode_workspace_size_ex(ctypes.byref(d), 1, 1, 3) == 0  # no such mode
