@@ -27,7 +27,7 @@
 //
 // Warp roles (224 threads, one CTA per SM, persistent, units taken from an
 // atomic ticket):
-//   warp 0      TMA producer (lane 0): nine [64][64] boxes per tile, 128 B swizzle
+//   warp 0      TMA producer: nine [64][64] boxes per tile, 128 B swizzle
 //   warp 1      TMEM allocation; lane 0 issues the S MMAs of each tile
 //   warps 2..5  softmax, lazy rescale of O^T, epilogue (one per TMEM lane
 //               quadrant; lanes l and l + 16 share head l's 64 tokens)
@@ -157,69 +157,101 @@ __global__ void __launch_bounds__(kThreads, 1)
 
     if (warp == 0) {
         // ------------------------------------------------------------------ producer
-        if (lane == 0) {
-            const uint64_t pol = l2_policy_evict_first();
-            tma_prefetch_desc(&tmC);
-            int stage = 0, issued = 0;
-            uint32_t phase = 0;
-            bool ok = true;
-            while (ok) {
-                const int ui = atomicAdd(a.ticket, 1);
-                const bool done = ui >= num_units;
-                Unit u;
-                int nt = 1;
-                if (!done) {
-                    u = a.units[ui];
-                    nt = (u.t1 - u.t0 + kT - 1) / kT;
+        // Nothing between a free stage and its tile's copies waits on global memory: the next
+        // unit (ticket, record, and the first 64 of its block-table entries) is fetched before
+        // the current one ends, and each lane holds one entry of the current 32-tile
+        // window of the unit, the following window loaded 32 tiles ahead.  Lanes 0..8 issue
+        // the tile's nine boxes at once.
+        const uint64_t pol = l2_policy_evict_first();
+        if (lane == 0) tma_prefetch_desc(&tmC);
+        struct Cursor {
+            int ui;      // unit index
+            Unit u;
+            int np;      // tiles with tokens (0 for an empty unit, which still yields one tile)
+            int w0, w1;  // this lane's block-table entry of the current / next 32-tile window
+        };
+        // block-table entry of tile i of unit c (-1 past its tiles or its table row)
+        auto entry = [&](const Cursor& c, int i) -> int { return i < c.np ? page_of(a, c.u.n, c.u.b, c.u.t0 / P + i) : -1; };
+        auto fetch = [&](Cursor& c) -> bool {
+            int t = 0;
+            if (lane == 0) t = atomicAdd(a.ticket, 1);
+            c.ui = __shfl_sync(0xffffffffu, t, 0);
+            if (c.ui >= num_units) return false;
+            c.u = a.units[c.ui];
+            c.np = (c.u.t1 - c.u.t0 + kT - 1) / kT;
+            c.w0 = entry(c, lane);
+            c.w1 = entry(c, 32 + lane);
+            return true;
+        };
+        // the next unit is fetched 2 tiles before the current one ends (early enough to hide
+        // the ticket -> record -> entries chain, late enough not to hold a unit another CTA
+        // could start)
+        constexpr int kAhead = 2;
+        Cursor cur, nxt;
+        bool have = fetch(cur);
+        bool fetched = false, have_nxt = false;
+        int k = 0, stage = 0, issued = 0;
+        uint32_t phase = 0;
+        while (true) {
+            int waited = 1;
+            if (lane == 0) waited = mbar_wait(bar + B_TILE_EMPTY + stage, phase ^ 1, s_abort, a.status);
+            if (!__shfl_sync(0xffffffffu, waited, 0)) break;
+            if (lane == 0) TRACE(14, issued);
+            if (!have) {
+                if (lane == 0) {
+                    tmeta[stage] = StageMeta{-1, 0, 0, 0};
+                    mbar_arrive(bar + B_TILE_FULL + stage);
                 }
-                int k = 0;
-                do {
-                    if (!mbar_wait(bar + B_TILE_EMPTY + stage, phase ^ 1, s_abort, a.status)) {
-                        ok = false;
-                        break;
-                    }
-                    TRACE(14, issued);
-                    if (done) {
-                        tmeta[stage] = StageMeta{-1, 0, 0, 0};
-                        mbar_arrive(bar + B_TILE_FULL + stage);
-                        ok = false;
-                        break;
-                    }
-                    const int t = u.t0 + k * kT;
-                    const int nvalid = nt == 0 ? 0 : min(u.t1 - t, kT);
-                    const int flags = (k == 0 ? kStageFirst : 0) | (k >= nt - 1 ? kStageLast : 0);
-                    int pg = -1;
-                    if (nt > 0) {
-                        pg = page_of(a, u.n, u.b, t / P);
-                        if (pg < 0) record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
-                    }
-                    tmeta[stage] = StageMeta{ui, t, flags | ((pg >= 0 ? nvalid : 0) << 8), k};
-                    if (pg >= 0) {
-                        mbar_arrive_expect_tx(bar + B_TILE_FULL + stage, kTileBytes);
-                        uint8_t* dst = sm + kOffTiles + (size_t)stage * kTileBytes;
-                        const int32_t row0 = pg * P + (t % P);
-#pragma unroll
-                        for (int kb = 0; kb < kKB; kb++)
-                            tma_load_2d(dst + kb * kBox, &tmC, kb * 64, row0, bar + B_TILE_FULL + stage, pol);
-                    } else {
-                        mbar_arrive(bar + B_TILE_FULL + stage);
-                    }
-                    TRACE(15, issued);
-                    issued++;
-                    if (++stage == kStages) {
-                        stage = 0;
-                        phase ^= 1;
-                    }
-                    k++;
-                } while (k < nt);
+                break;
             }
-            if (*s_abort) {  // bounded drain of copies still in flight
-                int n = issued < kStages ? issued : kStages;
-                for (int i = 0; i < n; i++) {
-                    stage = stage == 0 ? kStages - 1 : stage - 1;
-                    if (stage == kStages - 1) phase ^= 1;
-                    mbar_wait(bar + B_TILE_FULL + stage, phase, nullptr, a.status);
+            const int nt = max(1, cur.np);
+            const int t = cur.u.t0 + k * kT;
+            const int pg = __shfl_sync(0xffffffffu, cur.w0, k & 31);
+            const int nvalid = cur.np == 0 ? 0 : min(cur.u.t1 - t, kT);
+            const int flags = (k == 0 ? kStageFirst : 0) | (k == nt - 1 ? kStageLast : 0);
+            if (lane == 0) {
+                if (cur.np > 0 && pg < 0) record_status(a.status, DCP_ERR_UNALLOCATED_PAGE);
+                tmeta[stage] = StageMeta{cur.ui, t, flags | ((pg >= 0 ? nvalid : 0) << 8), k};
+            }
+            if (pg >= 0) {
+                if (lane == 0) mbar_arrive_expect_tx(bar + B_TILE_FULL + stage, kTileBytes);
+                __syncwarp();
+                if (lane < kKB)
+                    tma_load_2d(sm + kOffTiles + (size_t)stage * kTileBytes + lane * kBox, &tmC, lane * 64, pg * P,
+                                bar + B_TILE_FULL + stage, pol);
+            } else if (lane == 0) {
+                mbar_arrive(bar + B_TILE_FULL + stage);
+            }
+            if (lane == 0) TRACE(15, issued);
+            issued++;
+            if (++stage == kStages) {
+                stage = 0;
+                phase ^= 1;
+            }
+            // next tile: the next window of this unit, or the unit fetched ahead
+            ++k;
+            if (!fetched && nt - k <= kAhead) {
+                have_nxt = fetch(nxt);
+                fetched = true;
+            }
+            if (k < nt) {
+                if ((k & 31) == 0) {
+                    cur.w0 = cur.w1;
+                    cur.w1 = entry(cur, k + 32 + lane);
                 }
+            } else {
+                have = have_nxt;
+                fetched = false;
+                k = 0;
+                if (have) cur = nxt;
+            }
+        }
+        if (lane == 0 && *s_abort) {  // bounded drain of copies still in flight
+            int n = issued < kStages ? issued : kStages;
+            for (int i = 0; i < n; i++) {
+                stage = stage == 0 ? kStages - 1 : stage - 1;
+                if (stage == kStages - 1) phase ^= 1;
+                mbar_wait(bar + B_TILE_FULL + stage, phase, nullptr, a.status);
             }
         }
     } else if (warp == 1 || warp == 6) {
