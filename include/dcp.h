@@ -389,6 +389,28 @@ dcp_status dcp_merge(int32_t N, int32_t B, int32_t H, int32_t Dv, const float* o
  */
 dcp_status dcp_get_device_status(int32_t* status_out, void* stream);
 
+/*
+ * dcp_selftest_bounded_wait -- runs the failure path of the decode kernels'
+ * bounded waits, without a fault.  The persistent kernels wait on mbarriers
+ * (page copies landed, scores ready, buffers free) with a 4 s limit on the
+ * GPU's nanosecond timer; a wait that runs out records DCP_ERR_TIMEOUT in the
+ * sticky status word and raises its CTA's abort flag, and the kernel returns.
+ * In a correct run that never happens.  Here one thread waits, through the
+ * same code, on a barrier that nothing arrives on.  Not part of the method
+ * ("Efficient Decode Context Parallelism with vLLM for Long Context
+ * Workloads" has no counterpart); it exists so that the timeout path is
+ * exercised on a GPU.
+ *  result  DEVICE int64 [3], 16-byte aligned, caller-owned, written by the
+ *          kernel: [0] 1 if the wait reported completion (never expected),
+ *          [1] the abort flag after the wait (1 expected), [2] the
+ *          nanoseconds the wait took (at least the 4 s limit).
+ * Asynchronous on `stream` (about 4 s of one thread on one SM); afterwards
+ * dcp_get_device_status returns DCP_ERR_TIMEOUT (and clears it), and the
+ * context stays usable.  Returns DCP_ERR_INVALID_ARG for a NULL result,
+ * DCP_ERR_MISALIGNED for a misaligned one, DCP_ERR_CUDA if the launch fails.
+ */
+dcp_status dcp_selftest_bounded_wait(int64_t* result, void* stream);
+
 #ifdef __cplusplus
 }
 #endif

@@ -97,9 +97,11 @@ def lib() -> ctypes.CDLL:
         L.dcp_decode_partial_noalloc.argtypes = [D, i32, P, P, P, P, P]
         L.dcp_merge.argtypes = [i32, i32, i32, i32, P, P, P, P, P]
         L.dcp_get_device_status.argtypes = [ctypes.POINTER(i32), P]
+        L.dcp_selftest_bounded_wait.argtypes = [P, P]
         for name in ("dcp_shard_counts", "dcp_shard_map", "dcp_kv_append", "dcp_decode_partial",
                      "dcp_decode_partial_multi", "dcp_decode_merged", "dcp_decode_partial_noalloc", "dcp_merge",
-                     "dcp_get_device_status", "dcp_kv_append_rank", "dcp_decode_rank", "dcp_lse_rescale"):
+                     "dcp_get_device_status", "dcp_kv_append_rank", "dcp_decode_rank", "dcp_lse_rescale",
+                     "dcp_selftest_bounded_wait"):
             getattr(L, name).restype = ctypes.c_int
         _lib = L
     return _lib
@@ -220,6 +222,12 @@ def dcp_merge(o_partial, lse, out, lse_out=None, stream=None) -> None:
     N, B, H, Dv = o_partial.shape
     _check(lib().dcp_merge(N, B, H, Dv, _ptr(o_partial), _ptr(lse), _ptr(out), _ptr(lse_out), _stream(stream)),
            "dcp_merge")
+
+
+def dcp_selftest_bounded_wait(result, stream=None) -> None:
+    """Launches the bounded-wait self-test: result int64 [>= 3] on the device receives
+    (wait completed?, abort flag, nanoseconds waited); the status word then holds DCP_ERR_TIMEOUT."""
+    _check(lib().dcp_selftest_bounded_wait(_ptr(result), _stream(stream)), "dcp_selftest_bounded_wait")
 
 
 def dcp_get_device_status(stream=None) -> int:

@@ -9,6 +9,9 @@
 
 namespace dcp {
 
+// In selftest.cu; declared here rather than in kernels.h because only this entry point calls it.
+cudaError_t launch_selftest_bounded_wait(int* status, int64_t* result, cudaStream_t s);
+
 // Sticky status word, one per device context.
 static __device__ int g_status;
 
@@ -555,6 +558,15 @@ dcp_status dcp_lse_rescale(int32_t N, int32_t rank, int32_t B, int32_t H, int32_
         return DCP_ERR_INVALID_ARG;
     if (!aligned16(o) || !aligned16(o_rs)) return DCP_ERR_MISALIGNED;
     return cuda_err(launch_lse_rescale(N, rank, B, H, Dv, lse_all, o, o_rs, lse_out, (cudaStream_t)stream));
+}
+
+dcp_status dcp_selftest_bounded_wait(int64_t* result, void* stream) {
+    if (!result) return DCP_ERR_INVALID_ARG;
+    if (!aligned16(result)) return DCP_ERR_MISALIGNED;
+    int* status = nullptr;
+    dcp_status st = device_info(&status, nullptr);
+    if (st != DCP_OK) return st;
+    return cuda_err(launch_selftest_bounded_wait(status, result, (cudaStream_t)stream));
 }
 
 dcp_status dcp_get_device_status(int32_t* status_out, void* stream) {

@@ -191,3 +191,10 @@ def test_new_entry_points_host_validation_without_gpu():
     assert L.dcp_lse_rescale(2, 0, 1, 4, 6, A, A, A, None, None) == dcp.DCP_ERR_INVALID_ARG    # Dv % 4
     assert L.dcp_lse_rescale(2, 0, 1, 4, 64, A, A + 4, A, None, None) == dcp.DCP_ERR_MISALIGNED
     assert L.dcp_decode_workspace_size_ex(ctypes.byref(d), 1, 1, 3) == 0  # no such mode
+
+
+def test_selftest_bounded_wait_host_validation_without_gpu():
+    """The bounded-wait self-test checks its result pointer before touching the device."""
+    L = dcp.lib()
+    assert L.dcp_selftest_bounded_wait(None, None) == dcp.DCP_ERR_INVALID_ARG
+    assert L.dcp_selftest_bounded_wait(1024 + 8, None) == dcp.DCP_ERR_MISALIGNED
