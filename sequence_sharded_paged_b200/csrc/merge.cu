@@ -15,6 +15,7 @@ namespace dcp {
 namespace {
 
 constexpr int kMergeWarps = 8;
+constexpr int kMergeFast = 8;  // shard counts up to this take the path with all loads in flight
 
 __global__ void __launch_bounds__(32 * kMergeWarps)
     merge_kernel(int N, int64_t BH, int Dv, const float* __restrict__ o_part, const float* __restrict__ lse_part,
@@ -35,19 +36,48 @@ __global__ void __launch_bounds__(32 * kMergeWarps)
     for (int n = 0; n < N; n++) sum += expf(__ldg(lse_part + (int64_t)n * BH + row) - M);
     const float L = M + logf(sum);
     if (lane == 0 && lse_out) lse_out[row] = L;
-    for (int v = lane; v < nv; v += 32) {
-        float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
-        for (int n = 0; n < N; n++) {
-            const float ln = __ldg(lse_part + (int64_t)n * BH + row);
-            if (ln == -INFINITY) continue;
-            const float w = expf(ln - L);
-            const float4 x = __ldcs(reinterpret_cast<const float4*>(o_part + ((int64_t)n * BH + row) * Dv) + v);
-            acc.x = fmaf(w, x.x, acc.x);
-            acc.y = fmaf(w, x.y, acc.y);
-            acc.z = fmaf(w, x.z, acc.z);
-            acc.w = fmaf(w, x.w, acc.w);
+    if (N <= kMergeFast) {
+        // the row's weights once, then every shard's 16 bytes of a column block loaded before any
+        // is used, so that N loads per lane are in flight (a shard with weight 0 is not read)
+        float w[kMergeFast];
+#pragma unroll
+        for (int n = 0; n < kMergeFast; n++) {
+            const float ln = n < N ? __ldg(lse_part + (int64_t)n * BH + row) : -INFINITY;
+            w[n] = ln == -INFINITY ? 0.f : expf(ln - L);
         }
-        o[v] = acc;
+        for (int v = lane; v < nv; v += 32) {
+            float4 x[kMergeFast];
+#pragma unroll
+            for (int n = 0; n < kMergeFast; n++)
+                x[n] = w[n] != 0.f
+                           ? __ldcs(reinterpret_cast<const float4*>(o_part + ((int64_t)n * BH + row) * Dv) + v)
+                           : make_float4(0.f, 0.f, 0.f, 0.f);
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+#pragma unroll
+            for (int n = 0; n < kMergeFast; n++) {
+                if (w[n] == 0.f) continue;
+                acc.x = fmaf(w[n], x[n].x, acc.x);
+                acc.y = fmaf(w[n], x[n].y, acc.y);
+                acc.z = fmaf(w[n], x[n].z, acc.z);
+                acc.w = fmaf(w[n], x[n].w, acc.w);
+            }
+            o[v] = acc;
+        }
+    } else {
+        for (int v = lane; v < nv; v += 32) {
+            float4 acc = make_float4(0.f, 0.f, 0.f, 0.f);
+            for (int n = 0; n < N; n++) {
+                const float ln = __ldg(lse_part + (int64_t)n * BH + row);
+                if (ln == -INFINITY) continue;
+                const float w = expf(ln - L);
+                const float4 x = __ldcs(reinterpret_cast<const float4*>(o_part + ((int64_t)n * BH + row) * Dv) + v);
+                acc.x = fmaf(w, x.x, acc.x);
+                acc.y = fmaf(w, x.y, acc.y);
+                acc.z = fmaf(w, x.z, acc.z);
+                acc.w = fmaf(w, x.w, acc.w);
+            }
+            o[v] = acc;
+        }
     }
     if (discard) {  // the partials are scratch: drop their lines from L2 without writing them back
         __syncwarp();

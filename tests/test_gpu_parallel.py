@@ -7,7 +7,6 @@ filled from every position through dcp_kv_append_rank).  The all-gather is a
 stack of the ranks' LSEs and the reduce-scatter a sum of their reweighted
 blocks; no rank waits on another.  The real collectives run in
 test_parallel_cpu.py (gloo ranks) and, here, on a one-rank NCCL group."""
-import os
 import socket
 
 import numpy as np
