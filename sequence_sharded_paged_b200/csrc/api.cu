@@ -310,7 +310,8 @@ bool decode_geometry(int kind, int dtype, int hq, int hkv, int dk, int dv, int p
         g->ctas = num_sms;  // one CTA per SM (shared memory and the whole TMEM)
         g->granule = page_size;
         g->min_chunk = 2048;
-        g->units_per_cta = 16;
+        // fewer, longer chunks: every chunk boundary costs an epilogue and a split merge here
+        g->units_per_cta = 8;
         return true;
     }
     if (kind == DCP_MLA) {

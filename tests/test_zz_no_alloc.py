@@ -97,8 +97,8 @@ def test_noalloc_rejects_fp8_high_concurrency_shape(N):
 
 @pytest.mark.gpu
 def test_noalloc_shrunk_plan_against_oracle():
-    """64 heads, 8 shards and 380k tokens: the standard plan (2,368 target units,
-    2,048-token chunks) needs 621 MB of split area, so the no-alloc plan drops to
+    """64 heads, 8 shards and 380k tokens: the standard plan (1,184 target units,
+    2,048-token chunks) needs 311 MB of split area, so the no-alloc plan drops to
     one unit per CTA and cuts chunks of ~2,600 tokens instead.  Different units
     give different rounding, so this case is held to the oracle's bar rather than
     to bit-equality with dcp_decode_partial."""
